@@ -1,0 +1,343 @@
+// api.cu -- the C ABI declared in include/attn.h: argument validation,
+// TMA tensor-map encoding and kernel launches.  Nothing here allocates
+// device memory; the only device state is the per-device error word.
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "attn.h"
+#include "kernels.h"
+
+namespace attn {
+namespace {
+
+__device__ unsigned int g_error_word;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  int status = ATTN_OK;            // ATTN_OK, ATTN_E_DEVICE or ATTN_E_CUDA
+  unsigned int *err = nullptr;     // device address of g_error_word
+};
+DeviceState g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+// Per-device set-up: capability check and the error word's device address.
+int device_state(unsigned int **err) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_E_CUDA;
+  DeviceState &s = g_dev[dev];
+  std::call_once(s.once, [&s, dev] {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      s.status = ATTN_E_CUDA;
+      return;
+    }
+    if (major != 10) {
+      s.status = ATTN_E_DEVICE;
+      return;
+    }
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) {
+      s.status = ATTN_E_CUDA;
+      return;
+    }
+    s.err = static_cast<unsigned int *>(p);
+  });
+  *err = s.err;
+  return s.status;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 tensor map over a [rows, heads, d] row-major tensor: dims
+// (d, heads, rows), box (64, 1, box_rows), 128-byte swizzle.
+int encode_3d(CUtensorMap *map, const void *ptr, int d, int heads, long long rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return ATTN_E_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * heads * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
+}
+
+int check_threshold(float thr) {
+  if (!(thr >= 0.f && thr <= 1.f)) return ATTN_E_THRESHOLD;   // also rejects NaN
+  return ATTN_OK;
+}
+
+float thr_to_log2(float thr) {
+  return thr > 0.f ? (float)log2((double)thr) : -INFINITY;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_get_config(attn_config *cfg) {
+  if (!cfg) return ATTN_E_NULL;
+  cfg->prefill_block_m = kPrefillBlockM;
+  cfg->prefill_block_n = kPrefillBlockN;
+  cfg->skip_tile = kSkipTile;
+  cfg->decode_splits = kDecodeSplits;
+  cfg->decode_split_tile = kDecodeSplitTile;
+  cfg->decode_page_size = kPageSize;
+  cfg->smallseq_max_s_kv = kSmallSeqMaxKv;
+  return ATTN_OK;
+}
+
+const char *attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_E_NULL: return "ATTN_E_NULL";
+    case ATTN_E_ALIGN: return "ATTN_E_ALIGN";
+    case ATTN_E_HEADS: return "ATTN_E_HEADS";
+    case ATTN_E_HEAD_DIM: return "ATTN_E_HEAD_DIM";
+    case ATTN_E_THRESHOLD: return "ATTN_E_THRESHOLD";
+    case ATTN_E_PAGE_SIZE: return "ATTN_E_PAGE_SIZE";
+    case ATTN_E_SMALLSEQ: return "ATTN_E_SMALLSEQ";
+    case ATTN_E_SHAPE: return "ATTN_E_SHAPE";
+    case ATTN_E_WORKSPACE: return "ATTN_E_WORKSPACE";
+    case ATTN_E_SCALE: return "ATTN_E_SCALE";
+    case ATTN_E_CUDA: return "ATTN_E_CUDA";
+    case ATTN_E_DEVICE: return "ATTN_E_DEVICE";
+    case ATTN_E_TOO_LARGE: return "ATTN_E_TOO_LARGE";
+    default: return "ATTN_E_UNKNOWN";
+  }
+}
+
+int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int total_q, int total_k, int max_q, int max_k,
+                       int h_q, int h_kv, int d, int causal, float scale,
+                       float skip_threshold, uint32_t *skip_mask,
+                       unsigned long long *skip_counts,
+                       attn_bf16 *out, float *lse, attn_stream_t stream) {
+  if (batch < 0 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0) return ATTN_E_SHAPE;
+  if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (!isfinite(scale)) return ATTN_E_SCALE;
+  int rc = check_threshold(skip_threshold);
+  if (rc) return rc;
+  if (batch > 0 && (max_q <= 0 || total_q <= 0)) return ATTN_E_SHAPE;
+  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !out) return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_E_ALIGN;
+  if ((long long)max_q > (1ll << 24) || (long long)max_k > (1ll << 24)) return ATTN_E_TOO_LARGE;
+  unsigned int *err = nullptr;
+  rc = device_state(&err);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  PrefillParams p{};
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.out = out;
+  p.lse = lse;
+  p.skip_mask = skip_mask;
+  p.skip_counts = skip_counts;
+  p.batch = batch;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.max_q = max_q;
+  p.max_k = max_k;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.group = h_q / h_kv;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.qb_max = (max_q + kPrefillBlockM - 1) / kPrefillBlockM;
+  p.kt_max = (max_k + kSkipTile - 1) / kSkipTile;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.thr_log2 = thr_to_log2(skip_threshold);
+  p.err = err;
+
+  if (skip_mask) {
+    const size_t bits = (size_t)batch * p.qb_max * h_q * p.kt_max;
+    if (bits && cudaMemsetAsync(skip_mask, 0, align_up(bits, 32) / 8, st) != cudaSuccess)
+      return ATTN_E_CUDA;
+  }
+  if (skip_counts && cudaMemsetAsync(skip_counts, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    return ATTN_E_CUDA;
+  if (batch == 0) return ATTN_OK;
+
+  CUtensorMap qmap, kmap, vmap;
+  if (encode_3d(&qmap, q, d, h_q, total_q, kPrefillBlockM) ||
+      encode_3d(&kmap, k, d, h_kv, total_k, kPrefillBlockN) ||
+      encode_3d(&vmap, v, d, h_kv, total_k, kPrefillBlockN))
+    return ATTN_E_CUDA;
+  return launch_prefill(p, qmap, kmap, vmap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+}
+
+int attn_varlen_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                    int batch, int total_q, int total_k, int max_q, int max_k,
+                    int h_q, int h_kv, int d, int causal, float scale,
+                    attn_bf16 *out, float *lse, attn_stream_t stream) {
+  return attn_varlen_fwd_ex(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_q,
+                            max_k, h_q, h_kv, d, causal, scale, 0.f, nullptr, nullptr, out, lse,
+                            stream);
+}
+
+size_t attn_paged_decode_workspace_size(int batch, int h_q, int d) {
+  if (batch <= 0 || h_q <= 0 || d <= 0) return 256;
+  const size_t rows = (size_t)batch * h_q * kDecodeSplits;
+  return align_up(rows * d * sizeof(float), 256) + align_up(rows * 2 * sizeof(float), 256);
+}
+
+int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                         const int32_t *block_table, const int32_t *seq_lens,
+                         int batch, int num_pages, int max_pages_per_seq, int page_size,
+                         int h_q, int h_kv, int d, float skip_threshold, float scale,
+                         uint32_t *skip_mask, unsigned long long *skip_counts,
+                         attn_bf16 *out, float *lse,
+                         void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  if (batch < 0 || num_pages < 0 || max_pages_per_seq < 0) return ATTN_E_SHAPE;
+  if (page_size != kPageSize) return ATTN_E_PAGE_SIZE;
+  if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || h_q / h_kv > kMaxGroup) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (!isfinite(scale)) return ATTN_E_SCALE;
+  int rc = check_threshold(skip_threshold);
+  if (rc) return rc;
+  if (batch > 0 && (num_pages <= 0 || max_pages_per_seq <= 0)) return ATTN_E_SHAPE;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return ATTN_E_ALIGN;
+  if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_E_TOO_LARGE;
+  const bool sequential = skip_threshold > 0.f;
+  if (!sequential && batch > 0) {
+    if (!workspace) return ATTN_E_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_E_ALIGN;
+    if (workspace_bytes < attn_paged_decode_workspace_size(batch, h_q, d)) return ATTN_E_WORKSPACE;
+  }
+  unsigned int *err = nullptr;
+  rc = device_state(&err);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  DecodeParams p{};
+  p.q = q;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.out = out;
+  p.lse = lse;
+  const size_t rows = (size_t)batch * h_q * kDecodeSplits;
+  p.ws_o = static_cast<float *>(workspace);
+  p.ws_ml = workspace ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                   align_up(rows * d * sizeof(float), 256))
+                      : nullptr;
+  p.skip_mask = skip_mask;
+  p.skip_counts = skip_counts;
+  p.batch = batch;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.group = h_q / h_kv;
+  p.d = d;
+  p.num_pages = num_pages;
+  p.max_pages = max_pages_per_seq;
+  p.kt_max = (max_pages_per_seq * page_size + kSkipTile - 1) / kSkipTile;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.thr_log2 = thr_to_log2(skip_threshold);
+  p.sequential = sequential ? 1 : 0;
+  p.err = err;
+
+  if (skip_mask) {
+    const size_t bits = (size_t)batch * h_kv * p.kt_max;
+    if (bits && cudaMemsetAsync(skip_mask, 0, align_up(bits, 32) / 8, st) != cudaSuccess)
+      return ATTN_E_CUDA;
+  }
+  if (skip_counts && cudaMemsetAsync(skip_counts, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    return ATTN_E_CUDA;
+  if (batch == 0) return ATTN_OK;
+
+  CUtensorMap kmap, vmap;
+  const long long slots = (long long)num_pages * page_size;
+  if (encode_3d(&kmap, k_cache, d, h_kv, slots, kPageSize) ||
+      encode_3d(&vmap, v_cache, d, h_kv, slots, kPageSize))
+    return ATTN_E_CUDA;
+  return launch_decode(p, kmap, vmap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+}
+
+int attn_paged_decode(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                      const int32_t *block_table, const int32_t *seq_lens,
+                      int batch, int num_pages, int max_pages_per_seq, int page_size,
+                      int h_q, int h_kv, int d, float skip_threshold, float scale,
+                      attn_bf16 *out, float *lse,
+                      void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  return attn_paged_decode_ex(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages,
+                              max_pages_per_seq, page_size, h_q, h_kv, d, skip_threshold, scale,
+                              nullptr, nullptr, out, lse, workspace, workspace_bytes, stream);
+}
+
+int attn_smallseq_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                      const int32_t *cu_seqlens_kv, int batch, int total_kv, int h, int d,
+                      int max_s_kv, float scale, attn_bf16 *out, attn_bf16 *weights,
+                      attn_stream_t stream) {
+  if (batch < 0 || total_kv < 0) return ATTN_E_SHAPE;
+  if (h < 1) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (max_s_kv < 1 || max_s_kv > kSmallSeqMaxKv) return ATTN_E_SMALLSEQ;
+  if (!isfinite(scale)) return ATTN_E_SCALE;
+  if (!q || !k || !v || !cu_seqlens_kv || !out) return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_E_ALIGN;
+  if (weights && (reinterpret_cast<uintptr_t>(weights) & 1u)) return ATTN_E_ALIGN;
+  unsigned int *err = nullptr;
+  int rc = device_state(&err);
+  if (rc) return rc;
+  SmallSeqParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.cu = cu_seqlens_kv;
+  p.out = out;
+  p.weights = weights;
+  p.batch = batch;
+  p.total_kv = total_kv;
+  p.h = h;
+  p.d = d;
+  p.max_s_kv = max_s_kv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err;
+  return launch_smallseq(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+}
+
+int attn_get_last_device_error(attn_stream_t stream) {
+  unsigned int *err = nullptr;
+  int rc = device_state(&err);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_E_CUDA;
+  unsigned int host = 0;
+  if (cudaMemcpyFromSymbol(&host, g_error_word, sizeof(host)) != cudaSuccess) return ATTN_E_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ATTN_E_CUDA;
+  return (int)host;
+}
+
+}  // extern "C"

@@ -1,0 +1,170 @@
+// common.cuh -- device helpers shared by the attention kernels (sm_100a).
+//
+// Inline PTX for mbarriers, TMA tensor copies and tcgen05 (5th-generation
+// tensor cores with TMEM accumulators), bf16 packing, and the bounded waits
+// every kernel uses: no wait in this library spins forever; a wait that
+// gives up records ATTN_DEVERR_TIMEOUT in the error word and returns false.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "attn.h"
+
+#define ATTN_DEVICE __device__ __forceinline__
+
+namespace attn {
+
+// Iterations of mbarrier.try_wait before a wait gives up.  Each try_wait
+// blocks for a hardware-defined slice, so this bounds a wait at well over a
+// second while a healthy pipeline never comes close.
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------------------
+// error word
+// ---------------------------------------------------------------------------
+ATTN_DEVICE void raise_error(unsigned int *err, unsigned int bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 helpers
+// ---------------------------------------------------------------------------
+ATTN_DEVICE float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+ATTN_DEVICE float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+ATTN_DEVICE float bf16_to_f32(uint16_t x) { return __uint_as_float(uint32_t(x) << 16); }
+
+// Two floats -> packed bf16x2 (round to nearest even); `lo` lands in bits 0..15.
+ATTN_DEVICE uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+ATTN_DEVICE uint16_t f32_to_bf16(float x) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+  return r;
+}
+
+// 2^x on the MUFU unit.
+ATTN_DEVICE float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// warp reductions
+// ---------------------------------------------------------------------------
+ATTN_DEVICE float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+ATTN_DEVICE float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory addresses, mbarriers
+// ---------------------------------------------------------------------------
+ATTN_DEVICE uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+ATTN_DEVICE void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+ATTN_DEVICE void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+ATTN_DEVICE void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+ATTN_DEVICE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+ATTN_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete.
+ATTN_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+  }
+  raise_error(err, ATTN_DEVERR_TIMEOUT);
+  return false;
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), no multicast anywhere in this library
+// ---------------------------------------------------------------------------
+ATTN_DEVICE void tma_prefetch_desc(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 3-D tiled load: coordinates (x innermost).  x * element size must be a
+// multiple of 16 bytes (callers only pass x = 0 or x = 64 bf16 elements).
+ATTN_DEVICE void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                             int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Same with an L2 eviction hint (cache policy from createpolicy).
+ATTN_DEVICE void tma_load_3d_hint(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                                  int x, int y, int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
+ATTN_DEVICE uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+ATTN_DEVICE uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a tile that a
+// TMA copy wrote with 128-byte swizzling (rows of 128 bytes, 1024-byte aligned
+// tile base): the chunk index is XORed with the row index modulo 8.
+ATTN_DEVICE uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
+  return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+ATTN_DEVICE uint32_t elect_lane0() { return (threadIdx.x & 31u) == 0u; }
+
+}  // namespace attn

@@ -1,0 +1,65 @@
+// kernels.h -- launch parameters shared between the C-ABI layer (api.cu) and
+// the kernel translation units.  Internal; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace attn {
+
+// Fixed geometry of this build.
+constexpr int kPrefillBlockM = 128;   // query rows per tcgen05 tile
+constexpr int kPrefillBlockN = 128;   // keys per S = Q K^T MMA tile
+constexpr int kSkipTile = 32;         // keys per skip-softmax unit
+constexpr int kDecodeSplits = 32;     // dense decode schedule: KV splits
+constexpr int kDecodeSplitTile = 128; // dense decode schedule: keys per tile
+constexpr int kPageSize = 16;
+constexpr int kSmallSeqMaxKv = 16;
+constexpr int kMaxGroup = 16;         // largest h_q / h_kv supported by decode
+
+struct SmallSeqParams {
+  const uint16_t *q, *k, *v;
+  const int32_t *cu;
+  uint16_t *out, *weights;
+  int batch, total_kv, h, d, max_s_kv;
+  float scale_log2;
+  unsigned int *err;
+};
+
+struct DecodeParams {
+  const uint16_t *q;            // [B, h_q, d]
+  const int32_t *block_table;   // [B, max_pages]
+  const int32_t *seq_lens;      // [B]
+  uint16_t *out;                // [B, h_q, d]
+  float *lse;                   // [B, h_q] or null
+  float *ws_o;                  // [B, h_q, splits, d]   (dense schedule)
+  float *ws_ml;                 // [B, h_q, splits, 2]   (dense schedule)
+  uint32_t *skip_mask;          // or null
+  unsigned long long *skip_counts;  // or null
+  int batch, h_q, h_kv, group, d, num_pages, max_pages, kt_max;
+  float scale_log2;             // scale * log2(e)
+  float thr_log2;               // log2(threshold); -inf when skipping is off
+  int sequential;               // 1: one split walking 32-key tiles (skip mode)
+  unsigned int *err;
+};
+
+struct PrefillParams {
+  const int32_t *cu_q, *cu_k;
+  uint16_t *out;
+  float *lse;
+  uint32_t *skip_mask;
+  unsigned long long *skip_counts;
+  int batch, total_q, total_k, max_q, max_k, h_q, h_kv, group, d, causal;
+  int qb_max, kt_max;           // ceil(max_q / 128), ceil(max_k / 32)
+  float scale_log2, thr_log2;
+  unsigned int *err;
+};
+
+cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                          cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap,
+                           const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t stream);
+
+}  // namespace attn

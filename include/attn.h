@@ -1,0 +1,246 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) fused attention-forward library.
+ *
+ * Three operations, all computing masked softmax(Q K^T * scale) V with an
+ * online (flash-attention style) softmax:
+ *
+ *   attn_varlen_fwd     packed variable-length GQA prefill, causal or not
+ *                       (NVIDIA/Model-Optimizer PR 1034, "Add Triton unified
+ *                       attention kernel with HuggingFace integration":
+ *                       variable-length batching, GQA, causal/non-causal).
+ *   attn_paged_decode   one query token per sequence against a paged KV cache
+ *                       (NVIDIA/Model-Optimizer PR 1941, "Add split-k decode
+ *                       kernel for skip softmax": a 32-split schedule of
+ *                       128-token tiles when skip-softmax is off, one
+ *                       sequential split of 32-token tiles when it is on).
+ *   attn_smallseq_fwd   s_q = 1, s_kv <= 16 cross attention over a huge batch,
+ *                       also returning the attention weights
+ *                       (ROCm/TransformerEngine PR 461, "Integrate CK varlen
+ *                       cross attention for small-seq (s_q=1, s_kv<=16)").
+ *
+ * Skip-softmax (NVIDIA/TensorRT-LLM PR 9821, "Skip Softmax Attention"):
+ * keys are visited in 32-key tiles in increasing order; a tile is skipped for
+ * a group of query rows when, for every row of the group,
+ * exp(tile_max - running_max) < skip_threshold.  A skipped tile contributes
+ * nothing to the output or its normaliser.  The threshold is a runtime float
+ * in [0, 1]; 0 disables skipping.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE memory owned by the caller; the library
+ *    allocates nothing and keeps no pointer after the call returns.
+ *  - bf16 tensors are passed as attn_bf16 (raw 16-bit patterns), row-major,
+ *    contiguous, base pointers 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    only enqueues work on it and returns; nothing synchronises.
+ *  - scale: the softmax scale applied to Q.K; must be finite.  Pass
+ *    1/sqrt(d) for the usual scaling.
+ *  - Query head hq reads KV head hq / (h_q / h_kv) (consecutive grouping).
+ *  - Causal masking is bottom-right aligned: query row i of a sequence with
+ *    s_q queries and s_k keys sees keys j <= i + s_k - s_q.
+ *  - A query row with no visible key gets output 0 and LSE -inf.
+ *  - LSE outputs are float32 natural-log log-sum-exp of the scaled scores
+ *    over the kept keys.
+ *  - Host-checkable argument errors return a negative ATTN_E_* code and
+ *    launch nothing.  Errors that depend on device data (bad cu_seqlens,
+ *    block-table entries, over-long rows) set a bit in a per-device error
+ *    word (ATTN_DEVERR_*) and the affected unit writes zeros; read and clear
+ *    it with attn_get_last_device_error().
+ *  - All entry points are thread-safe; concurrent calls on different streams
+ *    share only the device error word.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+typedef uint16_t attn_bf16;
+typedef void *attn_stream_t; /* a cudaStream_t */
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_E_NULL = -1,        /* a required pointer is NULL                         */
+  ATTN_E_ALIGN = -2,       /* a tensor pointer is not 16-byte aligned            */
+  ATTN_E_HEADS = -3,       /* h_q or h_kv < 1, h_q % h_kv != 0, or group > 16    */
+  ATTN_E_HEAD_DIM = -4,    /* head dim d not 64 or 128                           */
+  ATTN_E_THRESHOLD = -5,   /* skip threshold NaN or outside [0, 1]               */
+  ATTN_E_PAGE_SIZE = -6,   /* page_size other than 16                            */
+  ATTN_E_SMALLSEQ = -7,    /* max_s_kv outside [1, 16]                           */
+  ATTN_E_SHAPE = -8,       /* negative size, or max length <= 0 with work to do  */
+  ATTN_E_WORKSPACE = -9,   /* workspace NULL or smaller than the query says      */
+  ATTN_E_SCALE = -10,      /* scale not finite                                   */
+  ATTN_E_CUDA = -11,       /* a CUDA call failed (launch, tensor-map encode ...) */
+  ATTN_E_DEVICE = -12,     /* current device is not compute capability 10.x      */
+  ATTN_E_TOO_LARGE = -13   /* a size exceeds a documented implementation limit   */
+};
+
+/* Bits of the per-device error word. */
+enum attn_device_error {
+  ATTN_DEVERR_CU_SEQLENS = 1u << 0,  /* cu_seqlens not monotone, or beyond total / max     */
+  ATTN_DEVERR_SEQ_LEN = 1u << 1,     /* decode seq_len < 0 or > max_pages_per_seq*page    */
+  ATTN_DEVERR_BLOCK_TABLE = 1u << 2, /* block-table entry outside [0, num_pages)          */
+  ATTN_DEVERR_SMALLSEQ_LEN = 1u << 3,/* small-seq row with s_kv > max_s_kv                */
+  ATTN_DEVERR_TIMEOUT = 1u << 4      /* a pipeline wait gave up (kernel returned early)   */
+};
+
+/* Compile-time tile geometry of this build (reported for the tests). */
+typedef struct attn_config {
+  int prefill_block_m;      /* query rows per prefill tile (tcgen05 M)            */
+  int prefill_block_n;      /* keys per prefill MMA tile                          */
+  int skip_tile;            /* keys per skip-softmax unit (prefill and decode)    */
+  int decode_splits;        /* KV splits of the dense decode schedule             */
+  int decode_split_tile;    /* keys per tile of the dense split schedule          */
+  int decode_page_size;     /* the only supported page size                       */
+  int smallseq_max_s_kv;    /* largest supported small-seq key count              */
+} attn_config;
+
+/* Fills *cfg; returns ATTN_OK (ATTN_E_NULL if cfg is NULL). */
+ATTN_API int attn_get_config(attn_config *cfg);
+
+/* Human-readable name of a status code (static string). */
+ATTN_API const char *attn_status_string(int status);
+
+/*
+ * attn_varlen_fwd -- packed varlen GQA attention forward (prefill).
+ *
+ *   q            [total_q, h_q, d]  bf16
+ *   k, v         [total_k, h_kv, d] bf16
+ *   cu_seqlens_q [batch + 1] int32, exclusive prefix sums, cu[0] = 0,
+ *                cu[batch] <= total_q   (same for cu_seqlens_k / total_k)
+ *   max_q, max_k upper bounds of the per-sequence lengths (size the grid);
+ *                a sequence longer than them sets ATTN_DEVERR_CU_SEQLENS
+ *   d            64 or 128
+ *   out          [total_q, h_q, d] bf16 (written for every row of every
+ *                sequence; rows outside [cu[0], cu[batch]) are untouched)
+ *   lse          [total_q, h_q] float32, may be NULL
+ *
+ * Returns ATTN_OK or an ATTN_E_* code (nothing launched on error).
+ */
+ATTN_API int attn_varlen_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                    int batch, int total_q, int total_k, int max_q, int max_k,
+                    int h_q, int h_kv, int d, int causal, float scale,
+                    attn_bf16 *out, float *lse, attn_stream_t stream);
+
+/*
+ * attn_varlen_fwd_ex -- attn_varlen_fwd with the skip-softmax tile rule.
+ *
+ * Units: (sequence b, q-head, q-block of prefill_block_m rows) x (key tile of
+ * skip_tile keys).  The rows a unit serves are the query rows of the block
+ * that belong to sequence b.  A unit is visited when at least one of its
+ * (row, key) pairs is unmasked.
+ *
+ *   skip_threshold  in [0, 1]; 0 gives exactly attn_varlen_fwd's result
+ *   skip_mask       NULL, or a bit array of
+ *                   batch * ceil(max_q / block_m) * h_q * ceil(max_k / skip_tile)
+ *                   bits (uint32 words, bit i of word w = unit 32w + i), unit
+ *                   index ((b * QB + r) * h_q + hq) * KT + t with
+ *                   QB = ceil(max_q / block_m), KT = ceil(max_k / skip_tile).
+ *                   Cleared by the call; a set bit marks a skipped unit.
+ *   skip_counts     NULL, or 2 uint64: {visited units, skipped units};
+ *                   cleared by the call.
+ */
+ATTN_API int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int total_q, int total_k, int max_q, int max_k,
+                       int h_q, int h_kv, int d, int causal, float scale,
+                       float skip_threshold, uint32_t *skip_mask,
+                       unsigned long long *skip_counts,
+                       attn_bf16 *out, float *lse, attn_stream_t stream);
+
+/*
+ * attn_paged_decode_workspace_size -- bytes of workspace attn_paged_decode
+ * needs for this shape (a pure host query; 0 is never returned for
+ * batch * h_q > 0).  The dense schedule keeps, per (sequence, q-head, split),
+ * the split's running max, running sum and unnormalised output in float32.
+ */
+ATTN_API size_t attn_paged_decode_workspace_size(int batch, int h_q, int d);
+
+/*
+ * attn_paged_decode -- one query token per sequence against a paged cache.
+ *
+ *   q              [batch, h_q, d] bf16
+ *   k_cache,
+ *   v_cache        [num_pages, page_size, h_kv, d] bf16; token t of sequence
+ *                  b lives in page block_table[b, t / page_size], slot
+ *                  t % page_size
+ *   block_table    [batch, max_pages_per_seq] int32; entries beyond a
+ *                  sequence's last page are never read
+ *   seq_lens       [batch] int32, 0 <= seq_lens[b] <= max_pages_per_seq*page_size
+ *   page_size      16
+ *   skip_threshold 0: dense split-KV schedule (32 splits of 128-key tiles per
+ *                  (sequence, kv-head)) followed by a log-sum-exp combine;
+ *                  > 0 (and <= 1): one sequential split per (sequence,
+ *                  kv-head) walking 32-key tiles; a tile is skipped when all
+ *                  h_q / h_kv query heads of the group vote skip.
+ *   out            [batch, h_q, d] bf16
+ *   lse            [batch, h_q] float32, may be NULL
+ *   workspace      device buffer of >= attn_paged_decode_workspace_size(...)
+ *                  bytes, 16-byte aligned (needed only when skip_threshold
+ *                  is 0; may be NULL otherwise)
+ */
+ATTN_API int attn_paged_decode(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                      const int32_t *block_table, const int32_t *seq_lens,
+                      int batch, int num_pages, int max_pages_per_seq, int page_size,
+                      int h_q, int h_kv, int d, float skip_threshold, float scale,
+                      attn_bf16 *out, float *lse,
+                      void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_paged_decode_ex -- attn_paged_decode plus skip-softmax reporting.
+ *
+ *   skip_mask    NULL, or a bit array of batch * h_kv * ceil(max_pages_per_seq
+ *                * page_size / skip_tile) bits, unit index (b * h_kv + hk) * KT + t;
+ *                cleared by the call.
+ *   skip_counts  NULL, or 2 uint64 {visited tiles, skipped tiles}; cleared.
+ */
+ATTN_API int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                         const int32_t *block_table, const int32_t *seq_lens,
+                         int batch, int num_pages, int max_pages_per_seq, int page_size,
+                         int h_q, int h_kv, int d, float skip_threshold, float scale,
+                         uint32_t *skip_mask, unsigned long long *skip_counts,
+                         attn_bf16 *out, float *lse,
+                         void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_smallseq_fwd -- one query per sequence, at most 16 keys each.
+ *
+ *   q              [batch, h, d] bf16 (batch = number of query tokens)
+ *   k, v           [total_kv, h, d] bf16
+ *   cu_seqlens_kv  [batch + 1] int32 prefix sums of the per-sequence key counts
+ *   max_s_kv       runtime upper bound of the key counts, 1..16; it is the last
+ *                  dimension of `weights`.  A row with more keys sets
+ *                  ATTN_DEVERR_SMALLSEQ_LEN and writes zeros.
+ *   out            [batch, h, d] bf16
+ *   weights        NULL, or [batch, h, 1, max_s_kv] bf16: the softmax
+ *                  probabilities, zero beyond the row's own key count
+ * Non-causal; h_q = h_kv = h.
+ */
+ATTN_API int attn_smallseq_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                      const int32_t *cu_seqlens_kv, int batch, int total_kv, int h, int d,
+                      int max_s_kv, float scale, attn_bf16 *out, attn_bf16 *weights,
+                      attn_stream_t stream);
+
+/*
+ * attn_get_last_device_error -- synchronises `stream`, then returns and
+ * clears the current device's error word (a mask of ATTN_DEVERR_* bits), or
+ * a negative ATTN_E_CUDA if the synchronisation itself failed.
+ */
+ATTN_API int attn_get_last_device_error(attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

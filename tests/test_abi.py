@@ -1,0 +1,136 @@
+"""The C-ABI library loads and exports what include/attn.h declares; host-side
+argument checks return their error codes (no GPU needed: every call below is
+rejected before any CUDA call)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def A():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_attn_build", os.path.join(ROOT, "attention_varlen_gqa_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import attention_varlen_gqa_b200
+    return attention_varlen_gqa_b200
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "attn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(A):
+    names = header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(A.lib, n), f"{n} declared in attn.h but not exported"
+    assert set(names) == set(A.EXPORTS), "binding and header disagree"
+
+
+def test_no_torch_in_signatures():
+    with open(os.path.join(ROOT, "include", "attn.h")) as f:
+        text = f.read()
+    code = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    for word in ("torch", "at::", "Tensor", "c10"):
+        assert word not in code, word
+
+
+def test_config(A):
+    cfg = A.attn_get_config()
+    assert cfg == dict(prefill_block_m=128, prefill_block_n=128, skip_tile=32, decode_splits=32,
+                       decode_split_tile=128, decode_page_size=16, smallseq_max_s_kv=16)
+    assert A.lib.attn_get_config(None) == -1
+
+
+def test_status_strings(A):
+    assert A.lib.attn_status_string(0) == b"ATTN_OK"
+    assert A.lib.attn_status_string(-5) == b"ATTN_E_THRESHOLD"
+    assert A.lib.attn_status_string(-99) == b"ATTN_E_UNKNOWN"
+
+
+def test_workspace_query(A):
+    def align(x):
+        return (x + 255) // 256 * 256
+    for B, h, d in ((64, 32, 128), (1, 1, 64), (7, 3, 128)):
+        rows = B * h * 32
+        assert A.attn_paged_decode_workspace_size(B, h, d) == align(rows * d * 4) + align(rows * 8)
+
+
+FAKE = 1 << 20          # a 16-byte aligned fake address, never dereferenced
+
+
+def varlen(A, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cq=FAKE, ck=FAKE, batch=2, tq=10, tk=10, mq=5, mk=5, hq=4, hkv=2,
+             d=64, causal=1, scale=0.125, thr=0.0, mask=None, counts=None, out=FAKE, lse=None, stream=None)
+    a.update(kw)
+    return A.lib.attn_varlen_fwd_ex(a["q"], a["k"], a["v"], a["cq"], a["ck"], a["batch"], a["tq"], a["tk"],
+                                    a["mq"], a["mk"], a["hq"], a["hkv"], a["d"], a["causal"], a["scale"],
+                                    a["thr"], a["mask"], a["counts"], a["out"], a["lse"], a["stream"])
+
+
+def test_varlen_argument_errors(A):
+    assert varlen(A, hq=3) == -3
+    assert varlen(A, hkv=0) == -3
+    assert varlen(A, d=96) == -4
+    assert varlen(A, thr=-0.1) == -5
+    assert varlen(A, thr=1.5) == -5
+    assert varlen(A, thr=float("nan")) == -5
+    assert varlen(A, scale=float("inf")) == -10
+    assert varlen(A, q=None) == -1
+    assert varlen(A, out=None) == -1
+    assert varlen(A, k=FAKE + 8) == -2
+    assert varlen(A, mq=0) == -8
+    assert varlen(A, batch=-1) == -8
+    assert varlen(A, mq=1 << 25, mk=1 << 25) == -13
+
+
+def decode(A, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, batch=2, pages=4, maxp=2, ps=16, hq=8, hkv=2, d=128,
+             thr=0.0, scale=0.1, mask=None, counts=None, out=FAKE, lse=None, ws=FAKE, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return A.lib.attn_paged_decode_ex(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["batch"], a["pages"],
+                                      a["maxp"], a["ps"], a["hq"], a["hkv"], a["d"], a["thr"], a["scale"],
+                                      a["mask"], a["counts"], a["out"], a["lse"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_decode_argument_errors(A):
+    assert decode(A, ps=32) == -6
+    assert decode(A, hq=7) == -3
+    assert decode(A, hq=64, hkv=2) == -3          # group of 32 > 16
+    assert decode(A, d=256) == -4
+    assert decode(A, thr=2.0) == -5
+    assert decode(A, scale=float("nan")) == -10
+    assert decode(A, bt=None) == -1
+    assert decode(A, ws=None) == -9
+    assert decode(A, wsb=100) == -9
+    assert decode(A, ws=FAKE + 4) == -2
+    assert decode(A, pages=0) == -8
+
+
+def smallseq(A, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu=FAKE, batch=3, tk=9, h=2, d=128, maxs=4, scale=0.1, out=FAKE, w=None,
+             stream=None)
+    a.update(kw)
+    return A.lib.attn_smallseq_fwd(a["q"], a["k"], a["v"], a["cu"], a["batch"], a["tk"], a["h"], a["d"],
+                                   a["maxs"], a["scale"], a["out"], a["w"], a["stream"])
+
+
+def test_smallseq_argument_errors(A):
+    assert smallseq(A, maxs=0) == -7
+    assert smallseq(A, maxs=17) == -7
+    assert smallseq(A, d=32) == -4
+    assert smallseq(A, h=0) == -3
+    assert smallseq(A, cu=None) == -1
+    assert smallseq(A, w=FAKE + 1) == -2
+    assert smallseq(A, scale=-math.inf) == -10
