@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention-forward hot path on B200.
+
+One step = one pass over every operation of the hot path, each on its own
+synthetic workload resident in HBM:
+  prefill   varlen GQA causal prefill, 8 sequences with lengths U[512, 8192]
+            (seed 0 -> 24 900 tokens), h_q=32, h_kv=8, d=128, fp32 LSE
+  decode    paged one-token decode, batch 64, KV lengths U[1024, 32768],
+            16-token pages from a permuted pool, h_q=32, h_kv=8, d=128,
+            dense 32-split schedule + LSE combine
+  smallseq  30 720 one-query sequences with s_kv from {2,4,6,8,12,16},
+            h=16, d=128, attention weights returned
+The headline `value` is the prefill throughput (TFLOP/s over the allowed
+(query, key) pairs); the decode and small-seq rows report HBM GB/s.  Every
+operation's inputs are larger than the 126 MB L2, so no flush is needed
+between steps.  The skip-softmax workload (4 x 16384 prefill, batch 32 x
+32768 decode, peaked sink/window keys) is measured after the timed steps at
+thresholds {0, 1e-3, 1e-2, 0.1} and reported with its skipped-unit fraction.
+
+Multi-GPU (torchrun, one rank per GPU): the operations are independent
+problems, so every rank runs the same step on its own seed (weak scaling, no
+data-path collective); timing is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle instead (bounded samples of the
+prefill workload on the host cores; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL_WORKLOAD = ("varlen GQA causal prefill bf16: 8 seqs, lengths U[512,8192] (seed 0), "
+                    "h_q=32, h_kv=8, d=128, fp32 LSE, threshold 0")
+METRIC = "prefill TFLOP/s & decode/small-seq HBM GB/s vs B200 peak; skipped-tile %"
+UNIT = "TFLOP/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip"], default="all",
+                    help="profiling aid: run a single operation (no JSON line)")
+    ap.add_argument("--no-skip", action="store_true", help="leave out the skip-softmax measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="leave out the CPU oracle baseline")
+    ap.add_argument("--small", action="store_true",
+                    help="profiling aid with --only: quarter-size decode / small-seq batches")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def prefill_flops(lens_q, lens_k, h_q, d, causal):
+    """4 * d * h_q * (allowed (query, key) pairs): QK^T and PV, 2 flops per MAC."""
+    pairs = 0
+    for sq, sk in zip(lens_q, lens_k):
+        if causal:
+            # row i sees min(sk, max(0, i + sk - sq + 1)) keys
+            for_rows = [min(sk, max(0, i + sk - sq + 1)) for i in range(sq)] if sq != sk else None
+            pairs += sum(for_rows) if for_rows is not None else sq * (sq + 1) // 2
+        else:
+            pairs += sq * sk
+    return 4.0 * d * h_q * pairs
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "attention_varlen_gqa_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, src_hash, units_key, units):
+    """Per-launch DRAM bytes from the committed ncu summary, scaled to this
+    launch's units; None when the kernel source changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)[kernel]
+    except Exception:
+        return None
+    if rec.get("source_sha") != src_hash:
+        return None
+    return rec["dram_bytes"] * units / rec[units_key]
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the prefill workload)
+# ---------------------------------------------------------------------------
+
+def oracle_slab(i, seed=0):
+    """Run the fp64 oracle on slab i of the prefill workload: slabs are the
+    (sequence, kv-head group) pairs, sequences taken longest first and cycled.
+    Returns (flops, seconds, sequence length)."""
+    import numpy as np
+
+    import oracle
+    import workloads as W
+    lens = W.gqa_prefill_lens(seed)
+    d, G = 128, 4
+    order = sorted(range(len(lens)), key=lambda b: -lens[b])
+    L = lens[order[i % len(order)]]
+    rng = np.random.default_rng(seed + i)
+    q = W.f32_to_bf16_bits(rng.standard_normal((L, G, d), dtype=np.float32))
+    k = W.f32_to_bf16_bits(rng.standard_normal((L, 1, d), dtype=np.float32))
+    v = W.f32_to_bf16_bits(rng.standard_normal((L, 1, d), dtype=np.float32))
+    t0 = time.perf_counter()
+    oracle.varlen_attention(q, k, v, [0, L], [0, L], G, 1, True, 1.0 / math.sqrt(d))
+    return prefill_flops([L], [L], G, d, True), time.perf_counter() - t0, L
+
+
+def oracle_sample(budget_s, seed=0):
+    """Oracle slabs in order until `budget_s` seconds of CPU time have passed.
+    Returns (flops, seconds, description, threads)."""
+    done, flops, t_total, i = [], 0.0, 0.0, 0
+    while t_total < budget_s and i < 64:
+        f, t, L = oracle_slab(i, seed)
+        flops += f
+        t_total += t
+        done.append(L)
+        i += 1
+    threads = len(os.sched_getaffinity(0))
+    desc = (f"fp64 oracle on {len(done)} (sequence, kv-head group) slabs of the prefill workload "
+            f"(lengths {done}, 4 q-heads each, causal, d=128)")
+    return flops, t_total, desc, threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+    per_step, lens_done = [], []
+    flops_total = 0.0
+    for s in range(args.warmup + args.steps):
+        f, t, L = oracle_slab(s)
+        if s >= args.warmup:
+            per_step.append(t)
+            flops_total += f
+            lens_done.append(L)
+    threads = len(os.sched_getaffinity(0))
+    desc = (f"fp64 oracle, one (sequence, kv-head group) slab of the prefill workload per step "
+            f"(4 q-heads, causal, d=128; sequence lengths {lens_done})")
+    secs = sum(per_step)
+    value = flops_total / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL_WORKLOAD, "sample": "bounded per step"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU path
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import attention_varlen_gqa_b200 as A
+    import workloads as W
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    seed = rank
+
+    # ---------------- inputs (device-resident) ----------------
+    want = {"prefill", "decode", "smallseq"} if args.only == "all" else {args.only}
+    ops = []
+    if "prefill" in want:
+        pre = W.gqa_prefill(seed=seed, where="device")
+        pre_cq = torch.from_numpy(pre["cu_seqlens_q"]).to(dev)
+        pre_ck = torch.from_numpy(pre["cu_seqlens_k"]).to(dev)
+        pre_out = torch.empty_like(pre["q"])
+        pre_lse = torch.empty(pre["q"].shape[:2], dtype=torch.float32, device=dev)
+        pre_flops = prefill_flops(pre["lens_q"], pre["lens_k"], 32, 128, True)
+
+        def do_prefill():
+            A.attn_varlen_fwd(pre["q"], pre["k"], pre["v"], pre_cq, pre_ck, pre["max_q"], pre["max_k"],
+                              causal=True, out=pre_out, lse=pre_lse)
+        ops.append(("prefill", do_prefill))
+
+    if "decode" in want:
+        dec_batch = 16 if args.small else 64
+        dec = W.paged_decode(W.decode_lens(seed, batch=dec_batch), seed=seed, where="device")
+        dec_bt = torch.from_numpy(dec["block_table"]).to(dev)
+        dec_sl = torch.from_numpy(dec["seq_lens"]).to(dev)
+        dec_out = torch.empty_like(dec["q"])
+        dec_lse = torch.empty(dec["q"].shape[:2], dtype=torch.float32, device=dev)
+        dec_ws = torch.empty(A.attn_paged_decode_workspace_size(dec_batch, 32, 128), dtype=torch.uint8,
+                             device=dev)
+        L = dec["seq_lens"].astype(np.int64)
+        dec_bytes = float(L.sum() * 8 * 128 * 2 * 2 + dec_batch * 32 * 128 * 2 * 2 + dec_batch * 32 * 4 +
+                          (-(-L // 16)).sum() * 4 + dec_batch * 4)
+
+        def do_decode():
+            A.attn_paged_decode(dec["q"], dec["k_cache"], dec["v_cache"], dec_bt, dec_sl, out=dec_out,
+                                lse=dec_lse, workspace=dec_ws)
+        ops.append(("decode", do_decode))
+
+    if "smallseq" in want:
+        ss = W.smallseq(seed=seed, batch=7680 if args.small else 30720, where="device")
+        ss_cu = torch.from_numpy(ss["cu_seqlens_kv"]).to(dev)
+        ss_out = torch.empty_like(ss["q"])
+        ss_w = torch.empty((ss["batch"], 16, 1, 16), dtype=torch.bfloat16, device=dev)
+        tk = int(ss["cu_seqlens_kv"][-1])
+        ss_bytes = float(ss["batch"] * 16 * 128 * 2 * 2 + tk * 16 * 128 * 2 * 2 + ss["batch"] * 16 * 16 * 2 +
+                         (ss["batch"] + 1) * 4)
+
+        def do_smallseq():
+            A.attn_smallseq_fwd(ss["q"], ss["k"], ss["v"], ss_cu, 16, out=ss_out, weights=ss_w)
+        ops.append(("smallseq", do_smallseq))
+
+    if args.only in ("prefill", "decode", "smallseq"):
+        fn = dict(ops)[args.only]
+        for _ in range(args.warmup + args.steps):
+            fn()
+        torch.cuda.synchronize()
+        assert A.attn_get_last_device_error() == 0
+        return
+    if args.only == "skip":
+        measure_skip(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
+        return
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- warm-up ----------------
+    for _ in range(args.warmup):
+        for _, fn in ops:
+            fn()
+    torch.cuda.synchronize()
+    assert A.attn_get_last_device_error() == 0
+
+    # ---------------- timed steps ----------------
+    ev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)] for name, _ in ops}
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(stream)
+    for s in range(args.steps):
+        for name, fn in ops:
+            a, b = ev[name][s]
+            a.record(stream)
+            fn()
+            b.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    per = {name: sum(a.elapsed_time(b) for a, b in ev[name]) / args.steps for name, _ in ops}
+    assert A.attn_get_last_device_error() == 0
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    total_ms = max_over_ranks(total_ms)
+    per = {k: max_over_ranks(v) for k, v in per.items()}
+    flops_all = sum_over_ranks(pre_flops)
+    dec_bytes_all = sum_over_ranks(dec_bytes)
+    ss_bytes_all = sum_over_ranks(ss_bytes)
+    value = flops_all / (per["prefill"] * 1e-3) / 1e12
+
+    # ---------------- end to end through the public API, host buffers ----------------
+    host = {n: torch.empty(pre[n].shape, dtype=pre[n].dtype, pin_memory=True) for n in ("q", "k", "v")}
+    for n in host:
+        host[n].copy_(pre[n])
+    h_cq = torch.from_numpy(pre["cu_seqlens_q"]).pin_memory()
+    h_ck = torch.from_numpy(pre["cu_seqlens_k"]).pin_memory()
+    h_out = torch.empty(pre_out.shape, dtype=pre_out.dtype, pin_memory=True)
+    h_lse = torch.empty(pre_lse.shape, dtype=torch.float32, pin_memory=True)
+    d_in = {n: torch.empty_like(pre[n]) for n in ("q", "k", "v")}
+    d_cq, d_ck = torch.empty_like(pre_cq), torch.empty_like(pre_ck)
+
+    def e2e_step():
+        for n in ("q", "k", "v"):
+            d_in[n].copy_(host[n], non_blocking=True)
+        d_cq.copy_(h_cq, non_blocking=True)
+        d_ck.copy_(h_ck, non_blocking=True)
+        o, l = A.attn_varlen_fwd(d_in["q"], d_in["k"], d_in["v"], d_cq, d_ck, pre["max_q"], pre["max_k"],
+                                 causal=True, out=pre_out, lse=pre_lse)
+        h_out.copy_(o, non_blocking=True)
+        h_lse.copy_(l, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in host) + 2 * h_cq.numel() * 4
+    d2h = h_out.numel() * 2 + h_lse.numel() * 4
+
+    skip = None
+    if not args.no_skip:
+        skip = measure_skip(A, W, torch, dev, seed, pk, reps=3)
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    src = source_hash("prefill.cu", "tcgen05.cuh", "common.cuh")
+    pre_tflops = pre_flops / (per["prefill"] * 1e-3) / 1e12
+    pre_traffic = recorded_traffic("prefill_gqa_causal_24900", src, "flops", pre_flops)
+    roofline = {"bound": "tensor", "achieved": pre_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
+                "frac": pre_tflops / pk["bf16"], "traffic": pre_traffic,
+                "peak_kind": f"{pk['src']} bf16 dense (burst)",
+                "frac_of_2250_datasheet": pre_tflops / 2250.0}
+    dec_gbs = dec_bytes / (per["decode"] * 1e-3) / 1e9
+    ss_gbs = ss_bytes / (per["smallseq"] * 1e-3) / 1e9
+    rows = {
+        "prefill": {"ms": per["prefill"], "tflops": pre_tflops, "flops": pre_flops,
+                    "frac_of_measured": pre_tflops / pk["bf16"], "frac_of_2250": pre_tflops / 2250.0,
+                    "lens": pre["lens_q"]},
+        "decode": {"ms": per["decode"], "gbs": dec_gbs, "bytes": dec_bytes,
+                   "frac_of_measured": dec_gbs / pk["hbm"], "frac_of_8000": dec_gbs / 8000.0,
+                   "workload": "batch 64, KV U[1024,32768] seed 0, page 16, h 32/8, d 128, 32 splits",
+                   "traffic": recorded_traffic("decode_dense_b64", source_hash("decode.cu", "common.cuh"),
+                                               "bytes", dec_bytes)},
+        "smallseq": {"ms": per["smallseq"], "gbs": ss_gbs, "bytes": ss_bytes,
+                     "frac_of_measured": ss_gbs / pk["hbm"], "frac_of_8000": ss_gbs / 8000.0,
+                     "workload": "30720 x s_kv{2..16} seed 0, h 16, d 128, + weights",
+                     "traffic": recorded_traffic("smallseq_b30720", source_hash("smallseq.cu", "common.cuh"),
+                                                 "bytes", ss_bytes)},
+    }
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        f, t, desc, threads = oracle_sample(12.0)
+        cpu = {"value": f / t / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": t}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PREFILL_WORKLOAD, "step": "prefill + paged decode + small-seq",
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "rows": rows,
+        "skip": skip,
+        "cpu_baseline": cpu,
+        "e2e": {"value": pre_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "what": "prefill through attn_varlen_fwd with q/k/v/cu_seqlens copied from pinned host "
+                        "memory and out/lse copied back every step"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clock_info,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_skip(A, W, torch, dev, seed, pk, reps=3):
+    """Skip-softmax workload at thresholds {0, 1e-3, 1e-2, 0.1}."""
+    import numpy as np
+    res = {"prefill": {}, "decode": {}}
+    sp = W.skip_prefill(seed=seed, where="device")
+    cq = torch.from_numpy(sp["cu_seqlens_q"]).to(dev)
+    ck = torch.from_numpy(sp["cu_seqlens_k"]).to(dev)
+    out = torch.empty_like(sp["q"])
+    lse = torch.empty(sp["q"].shape[:2], dtype=torch.float32, device=dev)
+    counts = torch.zeros(2, dtype=torch.int64, device=dev)
+    dense_flops = prefill_flops(sp["lens_q"], sp["lens_k"], 32, 128, True)
+    for thr in (0.0, 1e-3, 1e-2, 0.1):
+        def run():
+            A.attn_varlen_fwd(sp["q"], sp["k"], sp["v"], cq, ck, sp["max_q"], sp["max_k"], causal=True,
+                              out=out, lse=lse, skip_threshold=thr, skip_counts=counts)
+        run()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        vis, sk = (int(x) for x in counts.tolist())
+        frac = sk / vis if vis and thr > 0 else 0.0
+        # executed: QK^T over visited units always, PV only over kept ones
+        executed = dense_flops * (1.0 - frac / 2.0)
+        res["prefill"][str(thr)] = {"ms": ms, "skipped_frac": frac, "visited_units": vis,
+                                    "skipped_units": sk,
+                                    "dense_equiv_tflops": dense_flops / ms / 1e9,
+                                    "executed_tflops_est": executed / ms / 1e9}
+    del sp, out, lse
+    sd = W.skip_decode(seed=seed, where="device")
+    bt = torch.from_numpy(sd["block_table"]).to(dev)
+    sl = torch.from_numpy(sd["seq_lens"]).to(dev)
+    dout = torch.empty_like(sd["q"])
+    dlse = torch.empty(sd["q"].shape[:2], dtype=torch.float32, device=dev)
+    ws = torch.empty(A.attn_paged_decode_workspace_size(32, 32, 128), dtype=torch.uint8, device=dev)
+    Ls = sd["seq_lens"].astype(np.int64)
+    kbytes = float(Ls.sum() * 8 * 128 * 2)
+    for thr in (0.0, 1e-3, 1e-2, 0.1):
+        def run():
+            A.attn_paged_decode(sd["q"], sd["k_cache"], sd["v_cache"], bt, sl, skip_threshold=thr,
+                                out=dout, lse=dlse, workspace=ws, skip_counts=counts)
+        run()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        vis, sk = (int(x) for x in counts.tolist())
+        frac = sk / vis if vis and thr > 0 else 0.0
+        alg = kbytes + kbytes * (1.0 - frac) + 32 * 32 * 128 * 2 * 2 + 32 * 32 * 4
+        res["decode"][str(thr)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
+                                   "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"]}
+    return res
+
+
+if __name__ == "__main__":
+    main()
