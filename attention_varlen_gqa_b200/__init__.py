@@ -38,6 +38,7 @@ EXPORTS = {
     "attn_paged_decode_workspace_size": (_S, [_I, _I, _I]),
     "attn_paged_decode": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _S, _P]),
     "attn_paged_decode_ex": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _P, _P, _S, _P]),
+    "attn_paged_decode_static": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P]),
     "attn_smallseq_fwd": (_I, [_P] * 4 + [_I] * 5 + [_F, _P, _P, _P]),
     "attn_get_last_device_error": (_I, [_P]),
 }
@@ -175,6 +176,38 @@ def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size=16, 
         _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
         _stream(stream))
     _check("attn_paged_decode", rc)
+    return out, lse
+
+
+STATIC_WORKSPACE_BYTES = 48 << 20
+
+
+def attn_paged_decode_static(q, k_cache, v_cache, block_table, seq_lens, page_size=16,
+                             skip_threshold=0.0, scale=None, out=None, lse=None, want_lse=True,
+                             stream=None):
+    """attn_paged_decode without a workspace argument, for callers that cannot
+    allocate device memory: the split partials live in the library's own
+    48 MiB device scratch array, shared by every call (calls that overlap on
+    the GPU race).  Output tensors may still be allocated here when not given."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    batch, h_q, d = q.shape
+    num_pages, ps, h_kv, _ = k_cache.shape
+    if ps != page_size:
+        raise ValueError(f"cache page dimension {ps} != page_size {page_size}")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((batch, h_q), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib.attn_paged_decode_static(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), batch, num_pages,
+        block_table.shape[1], page_size, h_q, h_kv, d, float(skip_threshold), scale, _ptr(out),
+        _ptr(lse), _stream(stream))
+    _check("attn_paged_decode_static", rc)
     return out, lse
 
 

@@ -295,6 +295,64 @@ int attn_paged_decode(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_b
                               nullptr, nullptr, out, lse, workspace, workspace_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace attn {
+namespace {
+
+// Scratch for attn_paged_decode_static: split-KV partials of callers that
+// cannot allocate.  Shared by every call on a device; see attn.h.
+static __device__ __align__(256) unsigned char g_static_workspace[ATTN_STATIC_WORKSPACE_BYTES];
+
+struct StaticScratch {
+  std::once_flag once;
+  cudaError_t status = cudaSuccess;
+  void *ptr = nullptr;
+};
+StaticScratch g_scratch[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device with that device current.  Host code must not pass the array's
+// name itself to a kernel: on the host it is only a stand-in symbol.
+int static_scratch(void **ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_E_CUDA;
+  StaticScratch &s = g_scratch[dev];
+  std::call_once(s.once, [&s] {
+    void *p = nullptr;
+    s.status = cudaGetSymbolAddress(&p, g_static_workspace);
+    s.ptr = (s.status == cudaSuccess) ? p : nullptr;
+  });
+  if (s.status != cudaSuccess || !s.ptr) return ATTN_E_CUDA;
+  *ptr = s.ptr;
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" {
+
+int attn_paged_decode_static(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                             const int32_t *block_table, const int32_t *seq_lens, int batch,
+                             int num_pages, int max_pages_per_seq, int page_size, int h_q, int h_kv,
+                             int d, float skip_threshold, float scale, attn_bf16 *out, float *lse,
+                             attn_stream_t stream) {
+  if (batch < 0 || h_q < 1 || d < 1) return ATTN_E_SHAPE;
+  if (attn_paged_decode_workspace_size(batch, h_q, d) > ATTN_STATIC_WORKSPACE_BYTES)
+    return ATTN_E_TOO_LARGE;
+  unsigned int *err = nullptr;
+  int rc = device_state(&err);
+  if (rc) return rc;
+  void *scratch = nullptr;
+  rc = static_scratch(&scratch);
+  if (rc) return rc;
+  return attn_paged_decode_ex(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages,
+                              max_pages_per_seq, page_size, h_q, h_kv, d, skip_threshold, scale,
+                              nullptr, nullptr, out, lse, scratch, ATTN_STATIC_WORKSPACE_BYTES,
+                              stream);
+}
+
 int attn_smallseq_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
                       const int32_t *cu_seqlens_kv, int batch, int total_kv, int h, int d,
                       int max_s_kv, float scale, attn_bf16 *out, attn_bf16 *weights,

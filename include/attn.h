@@ -214,6 +214,44 @@ ATTN_API int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, 
                          void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_paged_decode_static -- attn_paged_decode for callers that cannot
+ * allocate device memory.  (The source pages have no counterpart; this entry
+ * point exists only for such callers.)
+ *
+ * Some callers cannot hand the library a workspace: a serving runtime whose
+ * memory pool already owns the whole GPU and treats any further cudaMalloc
+ * as an error, or a plug-in interface that has no workspace argument and
+ * runs where a cudaMalloc (which may synchronise the device) is not
+ * allowed.  This variant takes the same arguments as attn_paged_decode minus
+ * the workspace and keeps the split-KV partials in a scratch array that the
+ * library itself holds in device memory:
+ *
+ *   - scratch limit: ATTN_STATIC_WORKSPACE_BYTES (48 MiB).  A shape whose
+ *     attn_paged_decode_workspace_size(batch, h_q, d) exceeds it returns
+ *     ATTN_E_TOO_LARGE and launches nothing (about batch * h_q <= 2900 at
+ *     d = 128, <= 5600 at d = 64).
+ *   - every GPU that loads the library reserves those 48 MiB until the
+ *     process exits.
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) for that device; make that first call before
+ *     any stream capture begins.
+ *   - all calls share the one array and it keeps whatever the last call left
+ *     in it (nothing there has to start at zero: every split writes its own
+ *     partial before the combine reads it).  Calls that can overlap on the
+ *     GPU -- on different streams without ordering between them -- race on
+ *     it and give wrong results; order them on one stream or use
+ *     attn_paged_decode with a workspace per stream.
+ *   - no cudaMalloc, cudaFree or other allocating routine is called.
+ */
+#define ATTN_STATIC_WORKSPACE_BYTES ((size_t)48 << 20)
+ATTN_API int attn_paged_decode_static(const attn_bf16 *q, const attn_bf16 *k_cache,
+                                      const attn_bf16 *v_cache, const int32_t *block_table,
+                                      const int32_t *seq_lens, int batch, int num_pages,
+                                      int max_pages_per_seq, int page_size, int h_q, int h_kv,
+                                      int d, float skip_threshold, float scale, attn_bf16 *out,
+                                      float *lse, attn_stream_t stream);
+
+/*
  * attn_smallseq_fwd -- one query per sequence, at most 16 keys each.
  *
  *   q              [batch, h, d] bf16 (batch = number of query tokens)
