@@ -143,7 +143,7 @@ int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *
   if (batch < 0 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0) return ATTN_E_SHAPE;
   if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0) return ATTN_E_HEADS;
   if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
-  if (!isfinite(scale)) return ATTN_E_SCALE;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
   int rc = check_threshold(skip_threshold);
   if (rc) return rc;
   if (batch > 0 && (max_q <= 0 || total_q <= 0)) return ATTN_E_SHAPE;
@@ -222,7 +222,7 @@ int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const att
   if (page_size != kPageSize) return ATTN_E_PAGE_SIZE;
   if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || h_q / h_kv > kMaxGroup) return ATTN_E_HEADS;
   if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
-  if (!isfinite(scale)) return ATTN_E_SCALE;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
   int rc = check_threshold(skip_threshold);
   if (rc) return rc;
   if (batch > 0 && (num_pages <= 0 || max_pages_per_seq <= 0)) return ATTN_E_SHAPE;
@@ -361,7 +361,7 @@ int attn_smallseq_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v
   if (h < 1) return ATTN_E_HEADS;
   if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
   if (max_s_kv < 1 || max_s_kv > kSmallSeqMaxKv) return ATTN_E_SMALLSEQ;
-  if (!isfinite(scale)) return ATTN_E_SCALE;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
   if (!q || !k || !v || !cu_seqlens_kv || !out) return ATTN_E_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_E_ALIGN;
   if (weights && (reinterpret_cast<uintptr_t>(weights) & 1u)) return ATTN_E_ALIGN;

@@ -55,7 +55,7 @@ ATTN_DEVICE uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
 //   (1 = bf16), 15 A major (0 = K), 16 B major (0 = K, 1 = MN),
 //   17-22 N >> 3, 24-28 M >> 4.
-constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
@@ -117,6 +117,16 @@ ATTN_DEVICE void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
 
 ATTN_DEVICE void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 ATTN_DEVICE void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Per-warpgroup register budget changes (all 128 threads of a warpgroup).
+template <uint32_t N>
+ATTN_DEVICE void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+ATTN_DEVICE void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 // Named barrier over a subset of the CTA's warps.
 ATTN_DEVICE void named_bar_sync(int id, int nthreads) {

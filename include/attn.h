@@ -33,7 +33,7 @@
  *    contiguous, base pointers 16-byte aligned.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *    only enqueues work on it and returns; nothing synchronises.
- *  - scale: the softmax scale applied to Q.K; must be finite.  Pass
+ *  - scale: the softmax scale applied to Q.K; must be finite and > 0.  Pass
  *    1/sqrt(d) for the usual scaling.
  *  - Query head hq reads KV head hq / (h_q / h_kv) (consecutive grouping).
  *  - Causal masking is bottom-right aligned: query row i of a sequence with
@@ -79,7 +79,7 @@ enum attn_status {
   ATTN_E_SMALLSEQ = -7,    /* max_s_kv outside [1, 16]                           */
   ATTN_E_SHAPE = -8,       /* negative size, or max length <= 0 with work to do  */
   ATTN_E_WORKSPACE = -9,   /* workspace NULL or smaller than the query says      */
-  ATTN_E_SCALE = -10,      /* scale not finite                                   */
+  ATTN_E_SCALE = -10,      /* scale not finite or not > 0                        */
   ATTN_E_CUDA = -11,       /* a CUDA call failed (launch, tensor-map encode ...) */
   ATTN_E_DEVICE = -12,     /* current device is not compute capability 10.x      */
   ATTN_E_TOO_LARGE = -13   /* a size exceeds a documented implementation limit   */

@@ -87,6 +87,8 @@ def test_varlen_argument_errors(A):
     assert varlen(A, thr=1.5) == -5
     assert varlen(A, thr=float("nan")) == -5
     assert varlen(A, scale=float("inf")) == -10
+    assert varlen(A, scale=0.0) == -10
+    assert varlen(A, scale=-0.5) == -10
     assert varlen(A, q=None) == -1
     assert varlen(A, out=None) == -1
     assert varlen(A, k=FAKE + 8) == -2
@@ -111,6 +113,7 @@ def test_decode_argument_errors(A):
     assert decode(A, d=256) == -4
     assert decode(A, thr=2.0) == -5
     assert decode(A, scale=float("nan")) == -10
+    assert decode(A, scale=0.0) == -10
     assert decode(A, bt=None) == -1
     assert decode(A, ws=None) == -9
     assert decode(A, wsb=100) == -9
