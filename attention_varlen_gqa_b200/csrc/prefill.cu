@@ -42,10 +42,10 @@ constexpr int kProducerWarp = 4 * kNQ;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kThreads = 384;                  // softmax warpgroups 0, 1; warpgroup 2: TMA, MMA, 2 idle
 // Register split: launched at 168 per thread (384 x 168 = 64 512), the
-// producer warpgroup gives back down to 72 and each softmax warpgroup grows
-// to 216: 2 x 128 x 216 + 128 x 72 = 64 512.
-constexpr uint32_t kRegsSoftmax = 216;
-constexpr uint32_t kRegsOther = 72;
+// producer / MMA warpgroup gives back down to 120 and each softmax warpgroup
+// grows to 192: 2 x 128 x 192 + 128 x 120 = 64 512 (no spills either side).
+constexpr uint32_t kRegsSoftmax = 192;
+constexpr uint32_t kRegsOther = 120;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
@@ -175,6 +175,62 @@ ATTN_DEVICE TileGeo tile_geo(const PrefillParams &p, const Seq &s, int r) {
   g.full_vis = p.causal ? min(s.s_k, g.r0 + diag + 1) : s.s_k;
   g.n = (g.active && g.k_end > 0) ? (g.k_end + BN - 1) / BN : 0;
   return g;
+}
+
+// ---------------------------------------------------------------------------
+// softmax pieces
+// ---------------------------------------------------------------------------
+// Of every 4 column pairs of a clean tile, this many take the FMA-pipe
+// polynomial for 2^x instead of MUFU ex2 (tiles with masked or skipped
+// entries use ex2 throughout, so those entries are exact zeros).
+constexpr int kEmuOf4 = 2;
+
+// Max of 32 consecutive entries starting at `base` (two independent chains).
+ATTN_DEVICE float max32(const float (&s)[128], int base) {
+  float a = max3(s[base], s[base + 1], s[base + 2]);
+  float b = max3(s[base + 3], s[base + 4], s[base + 5]);
+#pragma unroll
+  for (int c = base + 6; c < base + 30; c += 4) {
+    a = max3(a, s[c], s[c + 1]);
+    b = max3(b, s[c + 2], s[c + 3]);
+  }
+  return max3(a, b, fmaxf(s[base + 30], s[base + 31]));
+}
+
+// p = 2^(s * sl2 - mref) for the 128 entries of a row, written to TMEM as
+// bf16 pairs over the row's S columns; returns the row sum of p.
+template <bool MIX>
+ATTN_DEVICE float exp_rows_to_tmem(const float (&s)[128], float sl2, float mref, uint32_t tS) {
+  const uint64_t scale2 = f2_pack(sl2, sl2), neg_m2 = f2_pack(-mref, -mref);
+  uint64_t acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int e = 64 * h + 2 * c;
+      const uint64_t x = f2_fma(f2_pack(s[e], s[e + 1]), scale2, neg_m2);
+      uint64_t pr;
+      if (MIX && (c & 3) < kEmuOf4) {
+        pr = exp2_poly_x2(x);
+      } else {
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        pr = f2_pack(ex2(x0), ex2(x1));
+      }
+      acc[c & 3] = f2_add(acc[c & 3], pr);
+      float p0, p1;
+      f2_unpack(pr, p0, p1);
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32(tS + 32 * h, pk);
+  }
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float a, b;
+  f2_unpack(t, a, b);
+  return a + b;
 }
 
 // ---------------------------------------------------------------------------
@@ -435,7 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 128; ++c) s[c] = -INFINITY;
         }
         const int kbase = j * BN;
-        if (kbase + BN > g.full_vis) {            // the tile holds masked entries for some row
+        bool clean = kbase + BN <= g.full_vis;    // no masked entry in any row of the tile
+        if (!clean) {                             // the tile holds masked entries for some row
           const int lim = lim_row - kbase;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -448,10 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t my_votes = 0;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            float tmx = s[u * 32];
-#pragma unroll
-            for (int c = 1; c < 32; ++c) tmx = fmaxf(tmx, s[u * 32 + c]);
-            const float t2 = tmx * sl2;
+            const float t2 = max32(s, u * 32) * sl2;
             const bool vote = !row_valid || (t2 == -INFINITY) || (t2 - m_true < p.thr_log2);
             m_true = fmaxf(m_true, t2);
             my_votes |= uint32_t(vote) << u;
@@ -473,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 4; ++u) vis_bits |= uint32_t(kbase + 32 * u < g.k_end) << u;
           skip_bits &= vis_bits;
           pv_skip = ((skip_bits | ~vis_bits) & 15u) == 15u;
+          clean = clean && skip_bits == 0;
           if (quad == 0 && lane == 0) {
             n_vis += __popc(vis_bits);
             n_skip += __popc(skip_bits);
@@ -498,9 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             alive = false;
             break;
           }
-          float tmx = s[0];
-#pragma unroll
-          for (int c = 1; c < 128; ++c) tmx = fmaxf(tmx, s[c]);
+          const float tmx = fmaxf(fmaxf(max32(s, 0), max32(s, 32)), fmaxf(max32(s, 64), max32(s, 96)));
           m_true = fmaxf(m_true, tmx * sl2);
         }
 
@@ -511,19 +564,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_true;
         }
         const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-        float rs = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(s[64 * h + 2 * c], sl2, -mref));
-            const float p1 = ex2(fmaf(s[64 * h + 2 * c + 1], sl2, -mref));
-            rs += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(tS + 32 * h, pk);
-        }
+        const float rs = clean ? exp_rows_to_tmem<true>(s, sl2, mref, tS)
+                               : exp_rows_to_tmem<false>(s, sl2, mref, tS);
         l = l * alpha + rs;
         tmem_wait_st();
 
@@ -637,7 +679,28 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUte
   return cudaGetLastError();
 }
 
+__global__ void exp2_selftest_kernel(const float *x, float *y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    float a, b;
+    f2_unpack(exp2_poly_x2(f2_pack(x[i], x[i + 1])), a, b);
+    y[i] = a;
+    y[i + 1] = b;
+  } else if (i < n) {
+    float a, b;
+    f2_unpack(exp2_poly_x2(f2_pack(x[i], 0.f)), a, b);
+    y[i] = a;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_selftest(const float *x, float *y, int n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int pairs = (n + 1) / 2;
+  exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
                            const CUtensorMap &vmap, cudaStream_t stream) {
