@@ -406,9 +406,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         for (; k_issued < min(n, kSeqSlots); ++k_issued)
           issue_pages<D>(&kmap, slot_ptr(k_issued), &kfull[k_issued % kSeqSlots], pages,
                          (c0 + k_issued) * kChunk, L, hk, 0, 4, true);
-      float m_run[kMaxGroup];                         // running max per head (log2 units)
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) m_run[h] = -INFINITY;
+      // running max (log2 units) of head `lane` of the group, kept by lane
+      // `lane` of every warp (G <= 16 <= 32), so a vote is one warp ballot
+      float m_run = -INFINITY;
       uint32_t kept_bits = 0;                         // 2 bits per chunk: tiles A, B kept
 
       for (int i = 0; i < n + kSeqLookahead; ++i) {
@@ -443,14 +443,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           const bool vis_b = (c0 + i) * kChunk + kSkipTile < L;
 #pragma unroll
           for (int tt = 0; tt < 2; ++tt) {
-            bool all = true;
-            for (int h = 0; h < G; ++h) {
-              const float tm = fmaxf(qa_x[(2 * tt) * 16 + h], qa_x[(2 * tt + 1) * 16 + h]);
-              // a head votes skip when exp(tile max - running max) < threshold
-              all = all && ((tm == -INFINITY) || (tm - m_run[h] < p.thr_log2));
-              m_run[h] = fmaxf(m_run[h], tm);
-            }
-            keep[tt] = !all;
+            const bool head = ln.lane < G;
+            const float tm = head ? fmaxf(qa_x[(2 * tt) * 16 + ln.lane], qa_x[(2 * tt + 1) * 16 + ln.lane])
+                                  : -INFINITY;
+            // a head votes skip when exp(tile max - running max) < threshold
+            const bool vote = !head || (tm == -INFINITY) || (tm - m_run < p.thr_log2);
+            m_run = fmaxf(m_run, tm);
+            keep[tt] = !__all_sync(0xffffffffu, vote);
           }
           if (!vis_b) keep[1] = false;
           if (tid == 0) {
