@@ -104,6 +104,32 @@ def recorded_traffic(kernel, src_hash, units_key, units):
     return rec["dram_bytes"] * units / rec[units_key]
 
 
+def reduce_over_ranks(x, op, world, device):
+    """All-reduce one float over the ranks ("max" or "sum"); identity at world 1."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate_ranks(local, world, device):
+    """Whole-job figures from one rank's measurements.  Times are the max over
+    ranks (the slowest rank ends the step); work (FLOPs, bytes) is summed, since
+    every rank runs its own problems (weak scaling).  Every rank must call this
+    with the same keys in the same order: each key is one collective."""
+    out = {"per": {k: reduce_over_ranks(v, "max", world, device) for k, v in sorted(local["per"].items())}}
+    for k in ("total_ms", "e2e_ms"):
+        out[k] = reduce_over_ranks(local[k], "max", world, device)
+    for k in ("flops", "dec_bytes", "ss_bytes"):
+        out[k] = reduce_over_ranks(local[k], "sum", world, device)
+    out["value"] = out["flops"] / (out["per"]["prefill"] * 1e-3) / 1e12
+    out["e2e_value"] = out["flops"] / (out["e2e_ms"] * 1e-3) / 1e12
+    return out
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
 
@@ -344,27 +370,6 @@ def main():
     per = {name: sum(a.elapsed_time(b) for a, b in ev[name]) / args.steps for name, _ in ops}
     assert A.attn_get_last_device_error() == 0
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
-
-    total_ms = max_over_ranks(total_ms)
-    per = {k: max_over_ranks(v) for k, v in per.items()}
-    flops_all = sum_over_ranks(pre_flops)
-    dec_bytes_all = sum_over_ranks(dec_bytes)
-    ss_bytes_all = sum_over_ranks(ss_bytes)
-    value = flops_all / (per["prefill"] * 1e-3) / 1e12
-
     # ---------------- end to end through the public API, host buffers ----------------
     host = {n: torch.empty(pre[n].shape, dtype=pre[n].dtype, pin_memory=True) for n in ("q", "k", "v")}
     for n in host:
@@ -397,9 +402,11 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    e2e_ms_local = e0.elapsed_time(e1) / args.steps
     h2d = sum(host[n].numel() * host[n].element_size() for n in host) + 2 * h_cq.numel() * 4
     d2h = h_out.numel() * 2 + h_lse.numel() * 4
+    agg = aggregate_ranks({"per": per, "total_ms": total_ms, "e2e_ms": e2e_ms_local, "flops": pre_flops,
+                           "dec_bytes": dec_bytes, "ss_bytes": ss_bytes}, world, dev)
 
     skip = None
     if not args.no_skip:
@@ -410,6 +417,7 @@ def main():
             dist.destroy_process_group()
         return
 
+    # the roofline is per kernel launch on this GPU; `value` and the rows are whole-job
     src = source_hash("prefill.cu", "tcgen05.cuh", "common.cuh")
     pre_tflops = pre_flops / (per["prefill"] * 1e-3) / 1e12
     pre_traffic = recorded_traffic("prefill_gqa_causal_24900", src, "flops", pre_flops)
@@ -417,18 +425,19 @@ def main():
                 "frac": pre_tflops / pk["bf16"], "traffic": pre_traffic,
                 "peak_kind": f"{pk['src']} bf16 dense (burst)",
                 "frac_of_2250_datasheet": pre_tflops / 2250.0}
-    dec_gbs = dec_bytes / (per["decode"] * 1e-3) / 1e9
-    ss_gbs = ss_bytes / (per["smallseq"] * 1e-3) / 1e9
+    P = agg["per"]
+    dec_gbs = agg["dec_bytes"] / (P["decode"] * 1e-3) / 1e9 / world
+    ss_gbs = agg["ss_bytes"] / (P["smallseq"] * 1e-3) / 1e9 / world
     rows = {
-        "prefill": {"ms": per["prefill"], "tflops": pre_tflops, "flops": pre_flops,
-                    "frac_of_measured": pre_tflops / pk["bf16"], "frac_of_2250": pre_tflops / 2250.0,
-                    "lens": pre["lens_q"]},
-        "decode": {"ms": per["decode"], "gbs": dec_gbs, "bytes": dec_bytes,
+        "prefill": {"ms": P["prefill"], "tflops": agg["value"], "flops": agg["flops"],
+                    "frac_of_measured": agg["value"] / world / pk["bf16"],
+                    "frac_of_2250": agg["value"] / world / 2250.0, "lens": pre["lens_q"]},
+        "decode": {"ms": P["decode"], "gbs": dec_gbs * world, "bytes": agg["dec_bytes"],
                    "frac_of_measured": dec_gbs / pk["hbm"], "frac_of_8000": dec_gbs / 8000.0,
                    "workload": "batch 64, KV U[1024,32768] seed 0, page 16, h 32/8, d 128, 32 splits",
                    "traffic": recorded_traffic("decode_dense_b64", source_hash("decode.cu", "common.cuh"),
                                                "bytes", dec_bytes)},
-        "smallseq": {"ms": per["smallseq"], "gbs": ss_gbs, "bytes": ss_bytes,
+        "smallseq": {"ms": P["smallseq"], "gbs": ss_gbs * world, "bytes": agg["ss_bytes"],
                      "frac_of_measured": ss_gbs / pk["hbm"], "frac_of_8000": ss_gbs / 8000.0,
                      "workload": "30720 x s_kv{2..16} seed 0, h 16, d 128, + weights",
                      "traffic": recorded_traffic("smallseq_b30720", source_hash("smallseq.cu", "common.cuh"),
@@ -440,8 +449,8 @@ def main():
         cpu = {"value": f / t / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": t}
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": agg["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": agg["total_ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": PREFILL_WORKLOAD, "step": "prefill + paged decode + small-seq",
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
@@ -449,8 +458,8 @@ def main():
         "rows": rows,
         "skip": skip,
         "cpu_baseline": cpu,
-        "e2e": {"value": pre_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+        "e2e": {"value": agg["e2e_value"], "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": agg["e2e_ms"],
                 "what": "prefill through attn_varlen_fwd with q/k/v/cu_seqlens copied from pinned host "
                         "memory and out/lse copied back every step"},
         "gpu_launches": 4 * args.steps,
