@@ -191,6 +191,28 @@ ATTN_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps (it is woken when the phase completes, or after about `ns`
+// nanoseconds) instead of spinning, which leaves the issue slots of its SM
+// sub-partition to the warps that have work.
+ATTN_DEVICE bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+ATTN_DEVICE uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Bounded wait for the phase with the given parity to complete.
 ATTN_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
@@ -275,5 +297,17 @@ ATTN_DEVICE uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
 }
 
 ATTN_DEVICE uint32_t elect_lane0() { return (threadIdx.x & 31u) == 0u; }
+
+// One lane of a converged warp (elect.sync): the lane that issues a
+// single-thread instruction on the warp's behalf.
+ATTN_DEVICE bool elect_one() {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r));
+  return r != 0;
+}
 
 }  // namespace attn

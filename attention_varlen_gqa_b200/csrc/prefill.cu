@@ -20,11 +20,16 @@
 //                   2-stage ring (3-D tensor maps over the packed [tokens,
 //                   heads, d] tensors, 128-byte swizzle, GQA kv-head as a
 //                   coordinate).
-//   warp 9          TMEM owner and single-thread MMA issuer.  Per K/V tile j:
-//                   PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, so the tensor core works on
-//                   one tile while the other tile's softmax runs.
+//   warp 9          TMEM owner and MMA issuer (the warp runs the loop, one
+//                   elected lane issues).  Per K/V tile j: PV0_j, S0_{j+1},
+//                   PV1_j, S1_{j+1}, so the tensor core works on one tile while
+//                   the other tile's softmax runs; each P.V starts on keys
+//                   [0, 64) as soon as the softmax has written their P.
 //   warps 10-11     idle (they only complete the third warpgroup).
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Waiting warps sleep in mbarrier.try_wait instead of spinning: every SM
+// sub-partition hosts two softmax warps, and spinning waiters took issue
+// slots from the one computing exponentials.
 #include <math.h>
 
 #include "common.cuh"
@@ -50,6 +55,8 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "regi
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kDrainSpins = 1u << 20;
+constexpr uint32_t kSleepHintNs = 20000;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 template <int D>
 struct Smem {
@@ -58,8 +65,9 @@ struct Smem {
   static constexpr int kK = kQ + kNQ * kTile;
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kBar = kV + kStages * kTile;
-  // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], o_free[NQ]
-  static constexpr int kNumBars = 2 + 3 * kStages + 4 * kNQ;
+  // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], o_free[NQ],
+  // p_half[NQ]
+  static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kUsed = kMisc + 128;
   // at least ~116 KB so that a single CTA (and its 512 TMEM columns) owns an SM
@@ -84,9 +92,13 @@ ATTN_DEVICE void tie(uint32_t (&r)[32]) {
 // Bounded wait that also gives up when another role raised the abort flag.
 ATTN_DEVICE bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                unsigned int *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  // suspended waits, bounded both in time (one second) and in count
+  const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u && *abort_flag) return false;
+    if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
   }
   *abort_flag = 1;
   raise_error(err, ATTN_DEVERR_TIMEOUT);
@@ -180,14 +192,6 @@ ATTN_DEVICE TileGeo tile_geo(const PrefillParams &p, const Seq &s, int r) {
 // ---------------------------------------------------------------------------
 // softmax pieces
 // ---------------------------------------------------------------------------
-// Of every 4 column pairs of a clean tile, this many take the FMA-pipe
-// polynomial for 2^x instead of MUFU ex2 (tiles with masked or skipped
-// entries use ex2 throughout, so those entries are exact zeros).  Measured
-// on the 24 900-token GQA prefill: 0 -> 806, 1 -> 792, 2 -> 765 TFLOP/s; the
-// softmax is latency-bound rather than MUFU-bound in this kernel, so the
-// polynomial's extra instructions do not pay yet.
-constexpr int kEmuOf4 = 0;
-
 // Max of 32 consecutive entries starting at `base` (two independent chains).
 ATTN_DEVICE float max32(const float (&s)[128], int base) {
   float a = max3(s[base], s[base + 1], s[base + 2]);
@@ -200,40 +204,65 @@ ATTN_DEVICE float max32(const float (&s)[128], int base) {
   return max3(a, b, fmaxf(s[base + 30], s[base + 31]));
 }
 
-// p = 2^(s * sl2 - mref) for the 128 entries of a row, written to TMEM as
-// bf16 pairs over the row's S columns; returns the row sum of p.
-template <bool MIX>
-ATTN_DEVICE float exp_rows_to_tmem(const float (&s)[128], float sl2, float mref, uint32_t tS) {
+// -inf for the columns at or beyond `lim` (keys the row may not see).
+ATTN_DEVICE void mask_cols(uint32_t (&sr)[4][32], int lim) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if (c >= lim) sr[c >> 5][c & 31] = 0xff800000u;
+}
+
+ATTN_DEVICE float fmax3u(float m, uint32_t a, uint32_t b) {
+  return max3(m, __uint_as_float(a), __uint_as_float(b));
+}
+
+// Max of the 128 columns of a row (eight independent chains).
+ATTN_DEVICE float max128(const uint32_t (&sr)[4][32]) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const int e = 2 * c;
+    m[c & 7] = fmax3u(m[c & 7], sr[e >> 5][e & 31], sr[e >> 5][(e & 31) + 1]);
+  }
+  return fmaxf(fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5])), fmaxf(m[6], m[7]));
+}
+
+// p = 2^(s * sl2 - mref) for 64 columns of a row (32-column chunks a, b),
+// packed to bf16 pairs and stored to TMEM at `taddr` (32 columns); returns the
+// row sum of p as an f32x2 pair.  With MAX, the max of the 64 columns of
+// (c, d) and of (a, b) is taken alongside, on the ALU pipe while the
+// exponentials occupy MUFU.
+template <bool MAX>
+ATTN_DEVICE uint64_t exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
+                                   const uint32_t (&c)[32], const uint32_t (&d)[32], float sl2,
+                                   float mref, uint32_t taddr, float &tmx) {
   const uint64_t scale2 = f2_pack(sl2, sl2), neg_m2 = f2_pack(-mref, -mref);
   uint64_t acc[4];
+  float m[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = f2_pack(0.f, 0.f);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t pk[32];
+  for (int k = 0; k < 8; ++k) m[k] = -INFINITY;
+  uint32_t pk[32];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const int e = 64 * h + 2 * c;
-      const uint64_t x = f2_fma(f2_pack(s[e], s[e + 1]), scale2, neg_m2);
-      uint64_t pr;
-      if (MIX && (c & 3) < kEmuOf4) {
-        pr = exp2_poly_x2(x);
-      } else {
-        float x0, x1;
-        f2_unpack(x, x0, x1);
-        pr = f2_pack(ex2(x0), ex2(x1));
-      }
-      acc[c & 3] = f2_add(acc[c & 3], pr);
-      float p0, p1;
-      f2_unpack(pr, p0, p1);
-      pk[c] = pack_bf16x2(p0, p1);
+  for (int q = 0; q < 32; ++q) {
+    const int e = (2 * q) & 31;
+    const uint32_t x0u = q < 16 ? a[e] : b[e], x1u = q < 16 ? a[e + 1] : b[e + 1];
+    if (MAX) {
+      m[q & 3] = fmax3u(m[q & 3], x0u, x1u);
+      m[4 + (q & 3)] = fmax3u(m[4 + (q & 3)], q < 16 ? c[e] : d[e], q < 16 ? c[e + 1] : d[e + 1]);
     }
-    tmem_st32(tS + 32 * h, pk);
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(x0u), __uint_as_float(x1u)), scale2, neg_m2);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    acc[q & 3] = f2_add(acc[q & 3], f2_pack(p0, p1));
+    pk[q] = pack_bf16x2(p0, p1);
   }
-  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-  float a, b;
-  f2_unpack(t, a, b);
-  return a + b;
+  tmem_st32(taddr, pk);
+  if (MAX) tmx = fmaxf(fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5])), fmaxf(m[6], m[7]));
+  return f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
 }
 
 // ---------------------------------------------------------------------------
@@ -256,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *p_full = s_full + kNQ;
   uint64_t *o_done = p_full + kNQ;
   uint64_t *o_free = o_done + kNQ;
+  uint64_t *p_half = o_free + kNQ;              // P of keys [0, 64) of the tile is in TMEM
   uint32_t *misc = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   uint32_t *tmem_slot = misc;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
@@ -281,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[t], 4);
       mbar_init(&o_done[t], 1);
       mbar_init(&o_free[t], 4);
+      mbar_init(&p_half[t], 4);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -356,95 +387,126 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // =============== MMA issuer ===============
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
-      const uint32_t sQ = smem_u32(sm + L::kQ);
-      const uint32_t sK = smem_u32(sm + L::kK);
-      const uint32_t sV = smem_u32(sm + L::kV);
-      uint32_t kv_c = 0, q_c = 0;
-      uint32_t tile_c[kNQ] = {0, 0};   // tiles processed per query-tile slot (p_full / o_done phases)
-      uint32_t item_c[kNQ] = {0, 0};   // items with work per slot (o_free phases)
-      bool ok = true;
-
-      auto issue_s = [&](int t, uint32_t stage) {
+    // The whole warp runs the loop (waits, descriptor arithmetic) in
+    // convergent code; one elected lane issues each MMA and commit.  The warp
+    // shares its SM sub-partition with two busy softmax warps, so the
+    // per-MMA instruction count matters: descriptors are built once per
+    // group and stepped by constants (the 14-bit address field never
+    // carries: shared addresses are below 2^18).
+    const bool leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
+    constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
+    const uint32_t sQ = smem_u32(sm + L::kQ);
+    const uint32_t sK = smem_u32(sm + L::kK);
+    const uint32_t sV = smem_u32(sm + L::kV);
+    uint32_t kv_c = 0, q_c = 0;
+    uint32_t tile_c[kNQ] = {0, 0};   // tiles processed per query-tile slot (p_full / o_done phases)
+    uint32_t item_c[kNQ] = {0, 0};   // items with work per slot (o_free phases)
+    bool ok = true;
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, p.err));
+    };
+    auto commit = [&](uint64_t *bar) {
+      if (leader) tc_commit(bar);
+      __syncwarp();
+    };
+    auto issue_s = [&](int t, uint32_t stage) {
+      const uint64_t a0 = smem_desc_sw128(sQ + t * L::kTile, 16, 1024);
+      const uint64_t b0 = smem_desc_sw128(sK + stage * L::kTile, 16, 1024);
+      const uint32_t d = tmem + t * 128;
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(sQ + t * L::kTile + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + stage * L::kTile + off, 16, 1024);
-          mma_ss(tmem + t * 128, a, bd, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+          mma_ss(d, a0 + off, b0 + off, idS, kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[t]);
-      };
-
-      for (int k = 0, idx = sched_item(0); ok && idx < items; idx = sched_item(++k)) {
-        const Item it = item_at(p, idx);
-        const Seq sq = seq_at(p, it.b);
-        if (sq.bad) continue;
-        TileGeo g[kNQ];
-        int nmax = 0;
-        for (int t = 0; t < kNQ; ++t) {
-          g[t] = tile_geo(p, sq, it.r[t]);
-          nmax = max(nmax, g[t].n);
-        }
-        if (nmax == 0) continue;
-        if (!(ok = wait_or_abort(q_full, q_c & 1, abort_flag, p.err))) break;
-        if (!(ok = wait_or_abort(&k_full[kv_c % kStages], (kv_c / kStages) & 1, abort_flag, p.err))) break;
-        tc_fence_after();
-        for (int t = 0; t < kNQ; ++t)
-          if (g[t].n > 0) issue_s(t, kv_c % kStages);
-        uint32_t pv_started[kNQ] = {0, 0};
-        for (int j = 0; ok && j < nmax; ++j) {
-          const uint32_t c = kv_c + j, st = c % kStages;
-          bool v_ready = false, k_next_ready = false;
-          for (int t = 0; t < kNQ && ok; ++t) {
-            if (j >= g[t].n) continue;
-            if (!(ok = wait_or_abort(&p_full[t], tile_c[t] & 1, abort_flag, p.err))) break;
-            if (j == 0 && item_c[t] > 0 &&
-                !(ok = wait_or_abort(&o_free[t], (item_c[t] - 1) & 1, abort_flag, p.err)))
-              break;
-            tc_fence_after();
-            const bool skip = SKIP && skip_pv[t];
-            if (!skip) {
-              if (!v_ready) {
-                if (!(ok = wait_or_abort(&v_full[st], (c / kStages) & 1, abort_flag, p.err))) break;
-                tc_fence_after();
-                v_ready = true;
-              }
-#pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk) {
-                const uint64_t bd = smem_desc_sw128(sV + st * L::kTile + kk * 16 * 128, BN * 128, 1024);
-                mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bd, idPV,
-                       (kk > 0 || pv_started[t]) ? 1u : 0u);
-              }
-              pv_started[t] = 1;
-            }
-            tc_commit(&o_done[t]);
-            ++tile_c[t];
-            if (j + 1 < g[t].n) {
-              if (!k_next_ready) {
-                const uint32_t cn = c + 1;
-                if (!(ok = wait_or_abort(&k_full[cn % kStages], (cn / kStages) & 1, abort_flag, p.err)))
-                  break;
-                tc_fence_after();
-                k_next_ready = true;
-              }
-              issue_s(t, (c + 1) % kStages);
-            }
-          }
-          if (ok) tc_commit(&kv_empty[st]);
-        }
-        if (!ok) break;
-        tc_commit(q_empty);
-        for (int t = 0; t < kNQ; ++t) item_c[t] += g[t].n > 0 ? 1 : 0;
-        kv_c += nmax;
-        ++q_c;
       }
-      // every MMA must be complete before the TMEM is released
+      __syncwarp();
+    };
+
+    for (int k = 0, idx = sched_item(0); ok && idx < items; idx = sched_item(++k)) {
+      const Item it = item_at(p, idx);
+      const Seq sq = seq_at(p, it.b);
+      if (sq.bad) continue;
+      TileGeo g[kNQ];
+      int nmax = 0;
+#pragma unroll
+      for (int t = 0; t < kNQ; ++t) {
+        g[t] = tile_geo(p, sq, it.r[t]);
+        nmax = max(nmax, g[t].n);
+      }
+      if (nmax == 0) continue;
+      if (!(ok = wait_all(q_full, q_c & 1))) break;
+      if (!(ok = wait_all(&k_full[kv_c % kStages], (kv_c / kStages) & 1))) break;
+      tc_fence_after();
+#pragma unroll
       for (int t = 0; t < kNQ; ++t)
-        if (tile_c[t] > 0) drain(&o_done[t], (tile_c[t] - 1) & 1);
+        if (g[t].n > 0) issue_s(t, kv_c % kStages);
+      uint32_t pv_started[kNQ] = {0, 0};
+      for (int j = 0; ok && j < nmax; ++j) {
+        const uint32_t c = kv_c + j, st = c % kStages;
+        bool v_ready = false, k_next_ready = false;
+#pragma unroll
+        for (int t = 0; t < kNQ; ++t) {
+          if (!ok || j >= g[t].n) continue;
+          ok = wait_all(&p_half[t], tile_c[t] & 1);
+          if (ok && j == 0 && item_c[t] > 0) ok = wait_all(&o_free[t], (item_c[t] - 1) & 1);
+          if (!ok) continue;
+          tc_fence_after();
+          const bool skip = SKIP && skip_pv[t];
+          if (!skip) {
+            if (!v_ready) {
+              if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
+              tc_fence_after();
+              v_ready = true;
+            }
+            const uint64_t v0 = smem_desc_sw128(sV + st * L::kTile, BN * 128, 1024);
+            const uint32_t acc0 = pv_started[t];
+            const uint32_t d = tmem + 256 + t * 128, a = tmem + t * 128;
+            // keys [0, 64) as soon as their P is written, the rest after
+            if (leader) {
+#pragma unroll
+              for (int kk = 0; kk < BN / 32; ++kk)
+                mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, kk > 0 ? 1u : acc0);
+            }
+            __syncwarp();
+            if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) continue;
+            tc_fence_after();
+            if (leader) {
+#pragma unroll
+              for (int kk = BN / 32; kk < BN / 16; ++kk)
+                mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, 1u);
+            }
+            pv_started[t] = 1;
+          } else if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) {
+            continue;
+          }
+          commit(&o_done[t]);
+          ++tile_c[t];
+          if (j + 1 < g[t].n) {
+            if (!k_next_ready) {
+              const uint32_t cn = c + 1;
+              if (!(ok = wait_all(&k_full[cn % kStages], (cn / kStages) & 1))) continue;
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(t, (c + 1) % kStages);
+          }
+        }
+        if (ok) commit(&kv_empty[st]);
+      }
+      if (!ok) break;
+      commit(q_empty);
+#pragma unroll
+      for (int t = 0; t < kNQ; ++t) item_c[t] += g[t].n > 0 ? 1 : 0;
+      kv_c += nmax;
+      ++q_c;
     }
+    // every MMA must be complete before the TMEM is released
+#pragma unroll
+    for (int t = 0; t < kNQ; ++t)
+      if (tile_c[t] > 0) drain(&o_done[t], (tile_c[t] - 1) & 1);
   }
   } else {
     regs_increase<kRegsSoftmax>();
@@ -476,37 +538,119 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       bool pv_any = false;
 
-      for (int j = 0; j < g.n; ++j) {
-        // a failed wait anywhere turns the rest of the item into barrier-only
-        // iterations, so the warps never disagree about the named barrier below
-        bool ok = alive && wait_or_abort(&s_full[t], tile_c & 1, abort_flag, p.err);
-        ok = __all_sync(0xffffffffu, ok);
-        float s[128];
-        if (ok) {
-          tc_fence_after();
-          uint32_t sr[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tie(sr[c]);
-#pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = -INFINITY;
+      // One K/V tile of the dense (no skip) path.  From the second tile on,
+      // the exponentials of keys [0, 64) start at once against the current
+      // reference max while the tile max is taken alongside; only a row whose
+      // max grew past the lazy-rescale margin (after the first tile, rare)
+      // makes the warp redo them.  P of keys [0, 64) is handed to the MMA warp
+      // before the second half is computed, so the first half of P.V overlaps
+      // it.  The values written are those of computing the max first.
+      auto dense_step = [&](int j) -> bool {
+        const bool ok =
+            __all_sync(0xffffffffu, alive && wait_or_abort(&s_full[t], tile_c & 1, abort_flag, p.err));
+        if (!ok) {
+          alive = false;
+          return false;
         }
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tie(sr[c]);
         const int kbase = j * BN;
-        bool clean = kbase + BN <= g.full_vis;    // no masked entry in any row of the tile
-        if (!clean) {                             // the tile holds masked entries for some row
-          const int lim = lim_row - kbase;
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= lim) s[c] = -INFINITY;
+        if (kbase + BN > g.full_vis) mask_cols(sr, lim_row - kbase);
+        float mref = (m_used == -INFINITY) ? 0.f : m_used;
+        float tmx;
+        uint64_t rs0 = 0;
+        const bool spec = j > 0;
+        if (spec)
+          rs0 = exp64_to_tmem<true>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, tmx);
+        else
+          tmx = max128(sr);
+        m_true = fmaxf(m_true, tmx * sl2);
+        // lazy rescale: move the reference max only when it grew by more than 2^8
+        float alpha = 1.f;
+        const bool grow = m_true > m_used + kRescaleLog2 || (m_used == -INFINITY && m_true > -INFINITY);
+        if (grow) {
+          alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_true);
+          m_used = m_true;
+          mref = m_used;
         }
+        if (!spec || __any_sync(0xffffffffu, grow)) {
+          if (spec) tmem_wait_st();                 // the speculative half is overwritten
+          rs0 = exp64_to_tmem<false>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, tmx);
+        }
+        // rescale the O accumulator rows whose reference max moved
+        if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
+          const bool okw =
+              __all_sync(0xffffffffu, wait_or_abort(&o_done[t], (tile_c - 1) & 1, abort_flag, p.err));
+          if (!okw) alive = false;
+          if (okw) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_wait_ld();
+              tie(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_half[t]);
+        float unused;
+        const uint64_t rs1 = exp64_to_tmem<false>(sr[2], sr[3], sr[2], sr[3], sl2, mref, tS + 32, unused);
+        float ra, rb;
+        f2_unpack(f2_add(rs0, rs1), ra, rb);
+        l = l * alpha + (ra + rb);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[t]);
+        ++tile_c;
+        pv_any = true;
+        return alive;
+      };
 
-        bool pv_skip = false;
-        if (SKIP) {
+      for (int j = 0; j < g.n; ++j) {
+        if constexpr (!SKIP) {
+          if (!dense_step(j)) break;
+        } else {
+          // a failed wait anywhere turns the rest of the item into barrier-only
+          // iterations, so the warps never disagree about the named barrier below
+          bool ok = alive && wait_or_abort(&s_full[t], tile_c & 1, abort_flag, p.err);
+          ok = __all_sync(0xffffffffu, ok);
+          float s[128];
+          if (ok) {
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tie(sr[c]);
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = -INFINITY;
+          }
+          const int kbase = j * BN;
+          if (kbase + BN > g.full_vis) {            // the tile holds masked entries for some row
+            const int lim = lim_row - kbase;
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= lim) s[c] = -INFINITY;
+          }
+
+          bool pv_skip = false;
           // per 32-key sub-tile: vote skip when exp(tile max - running max) < threshold
           uint32_t my_votes = 0;
 #pragma unroll
@@ -533,7 +677,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 4; ++u) vis_bits |= uint32_t(kbase + 32 * u < g.k_end) << u;
           skip_bits &= vis_bits;
           pv_skip = ((skip_bits | ~vis_bits) & 15u) == 15u;
-          clean = clean && skip_bits == 0;
           if (quad == 0 && lane == 0) {
             n_vis += __popc(vis_bits);
             n_skip += __popc(skip_bits);
@@ -554,53 +697,56 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int c = 0; c < 32; ++c) s[u * 32 + c] = -INFINITY;
             }
-        } else {
-          if (!ok) {
-            alive = false;
-            break;
+
+          // lazy rescale: move the reference max only when it grew by more than 2^8
+          float alpha = 1.f;
+          if (m_true > m_used + kRescaleLog2 || (m_used == -INFINITY && m_true > -INFINITY)) {
+            alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_true);
+            m_used = m_true;
           }
-          const float tmx = fmaxf(fmaxf(max32(s, 0), max32(s, 32)), fmaxf(max32(s, 64), max32(s, 96)));
-          m_true = fmaxf(m_true, tmx * sl2);
-        }
-
-        // lazy rescale: move the reference max only when it grew by more than 2^8
-        float alpha = 1.f;
-        if (m_true > m_used + kRescaleLog2 || (m_used == -INFINITY && m_true > -INFINITY)) {
-          alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_true);
-          m_used = m_true;
-        }
-        const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-        const float rs = (kEmuOf4 > 0 && clean) ? exp_rows_to_tmem<true>(s, sl2, mref, tS)
-                                                : exp_rows_to_tmem<false>(s, sl2, mref, tS);
-        l = l * alpha + rs;
-        tmem_wait_st();
-
-        // rescale the O accumulator rows whose reference max moved
-        if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
-          const bool okw =
-              __all_sync(0xffffffffu, wait_or_abort(&o_done[t], (tile_c - 1) & 1, abort_flag, p.err));
-          if (!okw) alive = false;
-          if (okw) {
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tO + c * 32, o);
-              tmem_wait_ld();
-              tie(o);
+          const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+          // the same exponentials and row-sum order as the dense path, so a
+          // threshold that skips nothing reproduces it bit for bit
+          uint32_t sv[4][32];
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tO + c * 32, o);
+          for (int c = 0; c < 128; ++c) sv[c >> 5][c & 31] = __float_as_uint(s[c]);
+          float unused;
+          const uint64_t rs0 = exp64_to_tmem<false>(sv[0], sv[1], sv[0], sv[1], sl2, mref, tS, unused);
+          const uint64_t rs1 = exp64_to_tmem<false>(sv[2], sv[3], sv[2], sv[3], sl2, mref, tS + 32, unused);
+          float ra, rb;
+          f2_unpack(f2_add(rs0, rs1), ra, rb);
+          l = l * alpha + (ra + rb);
+          tmem_wait_st();
+
+          // rescale the O accumulator rows whose reference max moved
+          if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
+            const bool okw =
+                __all_sync(0xffffffffu, wait_or_abort(&o_done[t], (tile_c - 1) & 1, abort_flag, p.err));
+            if (!okw) alive = false;
+            if (okw) {
+              tc_fence_after();
+#pragma unroll 1
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld();
+                tie(o);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st32(tO + c * 32, o);
+              }
+              tmem_wait_st();
             }
-            tmem_wait_st();
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&p_half[t]);
+            mbar_arrive(&p_full[t]);
+          }
+          ++tile_c;
+          pv_any = pv_any || !pv_skip;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[t]);
-        ++tile_c;
-        if (!SKIP && !alive) break;
-        pv_any = pv_any || !pv_skip;
       }
       if (!alive) break;
 
