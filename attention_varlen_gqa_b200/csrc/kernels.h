@@ -54,6 +54,7 @@ struct PrefillParams {
   int qb_max, kt_max;           // ceil(max_q / 128), ceil(max_k / 32)
   float scale_log2, thr_log2;
   unsigned int *err;
+  int work_slot;                // work-claim counter of this launch (set by launch_prefill)
 };
 
 cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream);

@@ -32,6 +32,8 @@
 // slots from the one computing exponentials.
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
@@ -45,6 +47,15 @@ constexpr int kStages = 2;
 constexpr int kNQ = 2;                         // query tiles per work item
 constexpr int kProducerWarp = 4 * kNQ;
 constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kSchedWarp = kMmaWarp + 1;
+constexpr int kSchedDepth = 4;                 // work items claimed ahead
+constexpr int kSchedConsumers = 4 * kNQ + 2;   // warps that read each claimed item
+// Work-claim counters, one pair (next item, CTAs done) per launch slot; the
+// last CTA of a launch puts its pair back to zero.  Launches take slots in
+// turn, so up to kWorkSlots prefill launches may run at the same time on a
+// device.
+constexpr int kWorkSlots = 64;
+__device__ unsigned int g_work[kWorkSlots][2];
 constexpr int kThreads = 384;                  // softmax warpgroups 0, 1; warpgroup 2: TMA, MMA, 2 idle
 // Register split: launched at 168 per thread (384 x 168 = 64 512), the
 // producer / MMA warpgroup gives back down to 120 and each softmax warpgroup
@@ -66,8 +77,8 @@ struct Smem {
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kBar = kV + kStages * kTile;
   // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], o_free[NQ],
-  // p_half[NQ]
-  static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ;
+  // p_half[NQ], sched_full[SD], sched_empty[SD]
+  static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ + 2 * kSchedDepth;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kUsed = kMisc + 128;
   // at least ~116 KB so that a single CTA (and its 512 TMEM columns) owns an SM
@@ -286,17 +297,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *o_done = p_full + kNQ;
   uint64_t *o_free = o_done + kNQ;
   uint64_t *p_half = o_free + kNQ;              // P of keys [0, 64) of the tile is in TMEM
+  uint64_t *sched_full = p_half + kNQ;          // [kSchedDepth] a claimed item is in the ring
+  uint64_t *sched_empty = sched_full + kSchedDepth;
   uint32_t *misc = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   uint32_t *tmem_slot = misc;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
   volatile uint32_t *skip_pv = misc + 2;        // [kNQ]
   volatile uint32_t *votes = misc + 4;          // [kNQ][2][4]
+  volatile int *ring = reinterpret_cast<volatile int *>(misc + 20);   // [kSchedDepth] claimed items
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = num_items(p);
-  // k-th work item of this CTA: items are sorted heaviest first and dealt
-  // round-robin (a boustrophedon deal measured 3 % slower)
-  auto sched_item = [&](int k) { return k * (int)gridDim.x + (int)blockIdx.x; };
+  // Work items are numbered heaviest first.  A CTA starts on item blockIdx.x
+  // and then claims the next unclaimed one from the launch's counter (warp
+  // kSchedWarp, kSchedDepth items ahead), so CTAs that drew light items take
+  // more of them; the claimed item numbers reach every role through a ring in
+  // shared memory.  -1 ends the work.
+  auto pop_lane = [&](uint32_t n) -> int {      // single-thread roles
+    const uint32_t slot = n % kSchedDepth;
+    const int idx = wait_or_abort(&sched_full[slot], (n / kSchedDepth) & 1, abort_flag, p.err) ? ring[slot] : -1;
+    mbar_arrive(&sched_empty[slot]);
+    return idx;
+  };
+  auto pop_warp = [&](uint32_t n) -> int {      // whole-warp roles
+    const uint32_t slot = n % kSchedDepth;
+    const bool okw =
+        __all_sync(0xffffffffu, wait_or_abort(&sched_full[slot], (n / kSchedDepth) & 1, abort_flag, p.err));
+    const int idx = okw ? ring[slot] : -1;
+    __syncwarp();
+    if ((threadIdx.x & 31u) == 0u) mbar_arrive(&sched_empty[slot]);
+    return idx;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -312,6 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[t], 1);
       mbar_init(&o_free[t], 4);
       mbar_init(&p_half[t], 4);
+    }
+    for (int q = 0; q < kSchedDepth; ++q) {
+      mbar_init(&sched_full[q], 1);
+      mbar_init(&sched_empty[q], kSchedConsumers);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -335,13 +370,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t keep = policy_evict_last();     // K/V tiles are re-read by other q-heads
       uint32_t kv_c = 0, q_c = 0;
       bool ok = true;
-      for (int k = 0, idx = sched_item(0); ok && idx < items; idx = sched_item(++k)) {
+      for (uint32_t n = 0; ok; ++n) {
+        const int idx = pop_lane(n);
+        if (idx < 0) break;
         const Item it = item_at(p, idx);
         const Seq sq = seq_at(p, it.b);
-        if (sq.bad) {
-          raise_error(p.err, ATTN_DEVERR_CU_SEQLENS);
-          continue;
-        }
+        if (sq.bad) continue;
         TileGeo g[kNQ];
         int nmax = 0;
         for (int t = 0; t < kNQ; ++t) {
@@ -425,7 +459,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
 
-    for (int k = 0, idx = sched_item(0); ok && idx < items; idx = sched_item(++k)) {
+    for (uint32_t n = 0; ok; ++n) {
+      const int idx = pop_warp(n);
+      if (idx < 0) break;
       const Item it = item_at(p, idx);
       const Seq sq = seq_at(p, it.b);
       if (sq.bad) continue;
@@ -507,6 +543,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int t = 0; t < kNQ; ++t)
       if (tile_c[t] > 0) drain(&o_done[t], (tile_c[t] - 1) & 1);
+  } else if (warp == kSchedWarp) {
+    // =============== work claims ===============
+    if (lane == 0) {
+      unsigned int *next_item = &g_work[p.work_slot][0];
+      // an item holds work when one of its query tiles holds rows (a tile
+      // whose rows see no key still writes zeros and -inf); items of a
+      // sequence with broken cu_seqlens are reported and dropped here
+      auto has_work = [&](int idx) {
+        const Item it = item_at(p, idx);
+        const Seq sq = seq_at(p, it.b);
+        if (sq.bad) {
+          raise_error(p.err, ATTN_DEVERR_CU_SEQLENS);
+          return false;
+        }
+        bool any = false;
+#pragma unroll
+        for (int t = 0; t < kNQ; ++t) any = any || tile_geo(p, sq, it.r[t]).active;
+        return any;
+      };
+      int next = (int)blockIdx.x;
+      for (uint32_t n = 0;; ++n) {
+        while (next < items && !has_work(next)) next = (int)gridDim.x + (int)atomicAdd(next_item, 1u);
+        const uint32_t slot = n % kSchedDepth;
+        if (n >= kSchedDepth &&
+            !wait_or_abort(&sched_empty[slot], ((n / kSchedDepth) - 1) & 1, abort_flag, p.err))
+          break;
+        ring[slot] = next < items ? next : -1;
+        mbar_arrive(&sched_full[slot]);
+        if (next >= items) break;
+        next = (int)gridDim.x + (int)atomicAdd(next_item, 1u);
+      }
+    }
   }
   } else {
     regs_increase<kRegsSoftmax>();
@@ -523,7 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned long long n_vis = 0, n_skip = 0;
     bool alive = true;
 
-    for (int k = 0, idx = sched_item(0); alive && idx < items; idx = sched_item(++k)) {
+    for (uint32_t n = 0; alive; ++n) {
+      const int idx = pop_warp(n);
+      if (idx < 0) break;
       const Item it = item_at(p, idx);
       const Seq sq = seq_at(p, it.b);
       const TileGeo g = tile_geo(p, sq, it.r[t]);
@@ -804,6 +874,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  // every claim of this CTA is made; the last CTA to get here rearms the slot
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&g_work[p.work_slot][1], 1u) == gridDim.x - 1) {
+      atomicExch(&g_work[p.work_slot][0], 0u);
+      atomicExch(&g_work[p.work_slot][1], 0u);
+    }
+  }
 }
 
 int num_sms() {
@@ -827,7 +905,10 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUte
   const long long items = (p.group % 2 == 0) ? (long long)p.batch * p.qb_max * (p.h_q / 2)
                                              : (long long)p.batch * ((p.qb_max + 1) / 2) * p.h_q;
   const int grid = (int)(items < num_sms() ? items : num_sms());
-  prefill_kernel<D, SKIP><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, p);
+  static std::atomic<unsigned int> next_slot{0};
+  PrefillParams q = p;
+  q.work_slot = (int)(next_slot.fetch_add(1u) % kWorkSlots);
+  prefill_kernel<D, SKIP><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, q);
   return cudaGetLastError();
 }
 

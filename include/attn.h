@@ -125,6 +125,14 @@ ATTN_API const char *attn_status_string(int status);
  *                sequence; rows outside [cu[0], cu[batch]) are untouched)
  *   lse          [total_q, h_q] float32, may be NULL
  *
+ * Work balance: the kernel's CTAs claim work items from a counter the library
+ * keeps in device memory, one of 64 per device taken in turn by successive
+ * calls (attn_varlen_fwd and attn_varlen_fwd_ex alike) and re-zeroed by the
+ * kernel itself when it ends.  Up to 64 of these calls may therefore run
+ * concurrently on one device (on different streams, or as parallel branches
+ * of a CUDA graph); a 65th that overlaps them shares a counter and computes
+ * wrong rows.
+ *
  * Returns ATTN_OK or an ATTN_E_* code (nothing launched on error).
  */
 ATTN_API int attn_varlen_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,

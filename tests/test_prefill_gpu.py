@@ -207,3 +207,37 @@ def test_full_size_skip_prefill_sampled(A, thr):
     data = W.skip_prefill(seed=0, where="device")
     counts = _check_sampled(A, data, thr, [2], 3)
     assert int(counts[0]) > 0
+
+
+def test_concurrent_calls_and_counter_reuse(A):
+    """The kernel's CTAs claim work from a per-call counter (64 per device,
+    taken in turn and re-zeroed by the kernel).  Two calls in flight on two
+    streams, then more calls in a row than there are counters: every result
+    equals the first, single call's bit for bit."""
+    d1 = W.varlen_prefill([700, 300, 129, 1000], h_q=8, h_kv=2, d=128, causal=True, seed=21)
+    d2 = W.varlen_prefill([513, 64, 900], h_q=8, h_kv=2, d=128, causal=False, seed=22)
+    t1, t2 = _dev(d1), _dev(d2)
+
+    def call(d, t):
+        return A.attn_varlen_fwd(t["q"], t["k"], t["v"], t["cu_q"], t["cu_k"], d["max_q"], d["max_k"],
+                                 causal=d["causal"], scale=d["scale"])
+
+    r1, r2 = call(d1, t1), call(d2, t2)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for _ in range(4):
+        with torch.cuda.stream(s1):
+            o1 = call(d1, t1)
+        with torch.cuda.stream(s2):
+            o2 = call(d2, t2)
+        outs.append((o1, o2))
+    torch.cuda.synchronize()
+    for o1, o2 in outs:
+        assert torch.equal(o1[0], r1[0]) and torch.equal(o1[1], r1[1])
+        assert torch.equal(o2[0], r2[0]) and torch.equal(o2[1], r2[1])
+    again = [call(d1, t1) for _ in range(70)]
+    torch.cuda.synchronize()
+    for o in again:
+        assert torch.equal(o[0], r1[0]) and torch.equal(o[1], r1[1])
+    assert A.attn_get_last_device_error() == 0
