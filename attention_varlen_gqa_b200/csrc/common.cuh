@@ -213,10 +213,15 @@ ATTN_DEVICE uint64_t globaltimer_ns() {
   return t;
 }
 
-// Bounded wait for the phase with the given parity to complete.
+// Bounded wait for the phase with the given parity to complete: one plain
+// test, then suspended waits (woken by the phase completion), bounded by one
+// second of global time and by an iteration count.
 ATTN_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+    if (globaltimer_ns() - t0 > 1000000000ull) break;
   }
   raise_error(err, ATTN_DEVERR_TIMEOUT);
   return false;

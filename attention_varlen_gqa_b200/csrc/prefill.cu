@@ -77,9 +77,10 @@ struct Smem {
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kBar = kV + kStages * kTile;
   // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], o_free[NQ],
-  // p_half[NQ], sched_full[SD], sched_empty[SD]
-  static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ + 2 * kSchedDepth;
+  // p_half[NQ], sched_full[SD], sched_empty[SD], votes_ready[NQ][2]
+  static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ + 2 * kSchedDepth + 2 * kNQ;
   static constexpr int kMisc = kBar + kNumBars * 8;
+  static_assert(kMisc % 16 == 0, "the vote words are read as 16-byte vectors");
   static constexpr int kUsed = kMisc + 128;
   // at least ~116 KB so that a single CTA (and its 512 TMEM columns) owns an SM
   static constexpr int kBytes = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
@@ -203,16 +204,14 @@ ATTN_DEVICE TileGeo tile_geo(const PrefillParams &p, const Seq &s, int r) {
 // ---------------------------------------------------------------------------
 // softmax pieces
 // ---------------------------------------------------------------------------
-// Max of 32 consecutive entries starting at `base` (two independent chains).
-ATTN_DEVICE float max32(const float (&s)[128], int base) {
-  float a = max3(s[base], s[base + 1], s[base + 2]);
-  float b = max3(s[base + 3], s[base + 4], s[base + 5]);
-#pragma unroll
-  for (int c = base + 6; c < base + 30; c += 4) {
-    a = max3(a, s[c], s[c + 1]);
-    b = max3(b, s[c + 2], s[c + 3]);
-  }
-  return max3(a, b, fmaxf(s[base + 30], s[base + 31]));
+// AND of four consecutive 32-bit words in shared memory (16-byte aligned),
+// read with one volatile vector load.
+ATTN_DEVICE uint32_t and4_shared(const volatile uint32_t *p) {
+  uint32_t a, b, c, d;
+  asm volatile("ld.volatile.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(smem_u32(const_cast<const uint32_t *>(p))));
+  return a & b & c & d;
 }
 
 // -inf for the columns at or beyond `lim` (keys the row may not see).
@@ -226,28 +225,29 @@ ATTN_DEVICE float fmax3u(float m, uint32_t a, uint32_t b) {
   return max3(m, __uint_as_float(a), __uint_as_float(b));
 }
 
-// Max of the 128 columns of a row (eight independent chains).
-ATTN_DEVICE float max128(const uint32_t (&sr)[4][32]) {
-  float m[8];
+// Raw maxima of the four 32-column sub-tiles of a row (two chains each).
+ATTN_DEVICE void max_sub4(const uint32_t (&sr)[4][32], float (&um)[4]) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m[k] = -INFINITY;
+  for (int u = 0; u < 4; ++u) {
+    float a = -INFINITY, b = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
-    const int e = 2 * c;
-    m[c & 7] = fmax3u(m[c & 7], sr[e >> 5][e & 31], sr[e >> 5][(e & 31) + 1]);
+    for (int c = 0; c < 32; c += 4) {
+      a = fmax3u(a, sr[u][c], sr[u][c + 1]);
+      b = fmax3u(b, sr[u][c + 2], sr[u][c + 3]);
+    }
+    um[u] = fmaxf(a, b);
   }
-  return fmaxf(fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5])), fmaxf(m[6], m[7]));
 }
 
 // p = 2^(s * sl2 - mref) for 64 columns of a row (32-column chunks a, b),
-// packed to bf16 pairs and stored to TMEM at `taddr` (32 columns); returns the
-// row sum of p as an f32x2 pair.  With MAX, the max of the 64 columns of
-// (c, d) and of (a, b) is taken alongside, on the ALU pipe while the
-// exponentials occupy MUFU.
+// packed to bf16 pairs and stored to TMEM at `taddr` (32 columns); the sums
+// of p over chunk a and chunk b go to ps[0], ps[1].  With MAX, the raw maxima
+// of the four 32-column chunks a, b, c, d are taken alongside (on the ALU pipe
+// while the exponentials occupy MUFU) into um.
 template <bool MAX>
-ATTN_DEVICE uint64_t exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
-                                   const uint32_t (&c)[32], const uint32_t (&d)[32], float sl2,
-                                   float mref, uint32_t taddr, float &tmx) {
+ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
+                               const uint32_t (&c)[32], const uint32_t (&d)[32], float sl2, float mref,
+                               uint32_t taddr, float (&um)[4], float *ps) {
   const uint64_t scale2 = f2_pack(sl2, sl2), neg_m2 = f2_pack(-mref, -mref);
   uint64_t acc[4];
   float m[8];
@@ -261,19 +261,29 @@ ATTN_DEVICE uint64_t exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[
     const int e = (2 * q) & 31;
     const uint32_t x0u = q < 16 ? a[e] : b[e], x1u = q < 16 ? a[e + 1] : b[e + 1];
     if (MAX) {
-      m[q & 3] = fmax3u(m[q & 3], x0u, x1u);
-      m[4 + (q & 3)] = fmax3u(m[4 + (q & 3)], q < 16 ? c[e] : d[e], q < 16 ? c[e + 1] : d[e + 1]);
+      // chains 0-1: a, 2-3: b, 4-5: c, 6-7: d
+      const int ch = (q < 16 ? 0 : 2) + (q & 1);
+      m[ch] = fmax3u(m[ch], x0u, x1u);
+      m[4 + ch] = fmax3u(m[4 + ch], q < 16 ? c[e] : d[e], q < 16 ? c[e + 1] : d[e + 1]);
     }
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(x0u), __uint_as_float(x1u)), scale2, neg_m2);
     float x0, x1;
     f2_unpack(x, x0, x1);
     const float p0 = ex2(x0), p1 = ex2(x1);
-    acc[q & 3] = f2_add(acc[q & 3], f2_pack(p0, p1));
+    const int ac = (q < 16 ? 0 : 2) + (q & 1);
+    acc[ac] = f2_add(acc[ac], f2_pack(p0, p1));
     pk[q] = pack_bf16x2(p0, p1);
   }
   tmem_st32(taddr, pk);
-  if (MAX) tmx = fmaxf(fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5])), fmaxf(m[6], m[7]));
-  return f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  if (MAX) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) um[u] = fmaxf(m[2 * u], m[2 * u + 1]);
+  }
+  float x0, x1;
+  f2_unpack(f2_add(acc[0], acc[1]), x0, x1);
+  ps[0] = x0 + x1;
+  f2_unpack(f2_add(acc[2], acc[3]), x0, x1);
+  ps[1] = x0 + x1;
 }
 
 // ---------------------------------------------------------------------------
@@ -299,10 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *p_half = o_free + kNQ;              // P of keys [0, 64) of the tile is in TMEM
   uint64_t *sched_full = p_half + kNQ;          // [kSchedDepth] a claimed item is in the ring
   uint64_t *sched_empty = sched_full + kSchedDepth;
+  uint64_t *votes_ready = sched_empty + kSchedDepth;   // [kNQ][2] the four warps' votes are written
   uint32_t *misc = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   uint32_t *tmem_slot = misc;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
-  volatile uint32_t *skip_pv = misc + 2;        // [kNQ]
+  // skip votes of the four warps of a softmax warpgroup, per query tile and
+  // tile parity: bit u = every row of the warp votes to skip 32-key sub-tile u
   volatile uint32_t *votes = misc + 4;          // [kNQ][2][4]
   volatile int *ring = reinterpret_cast<volatile int *>(misc + 20);   // [kSchedDepth] claimed items
 
@@ -343,6 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[t], 1);
       mbar_init(&o_free[t], 4);
       mbar_init(&p_half[t], 4);
+      mbar_init(&votes_ready[2 * t], 4);
+      mbar_init(&votes_ready[2 * t + 1], 4);
     }
     for (int q = 0; q < kSchedDepth; ++q) {
       mbar_init(&sched_full[q], 1);
@@ -428,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // group and stepped by constants (the 14-bit address field never
     // carries: shared addresses are below 2^18).
     const bool leader = elect_one();
+    const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
     constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
     constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
     const uint32_t sQ = smem_u32(sm + L::kQ);
@@ -436,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t kv_c = 0, q_c = 0;
     uint32_t tile_c[kNQ] = {0, 0};   // tiles processed per query-tile slot (p_full / o_done phases)
     uint32_t item_c[kNQ] = {0, 0};   // items with work per slot (o_free phases)
+    unsigned long long n_vis = 0, n_skip = 0;
     bool ok = true;
     auto wait_all = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, p.err));
@@ -490,34 +506,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && j == 0 && item_c[t] > 0) ok = wait_all(&o_free[t], (item_c[t] - 1) & 1);
           if (!ok) continue;
           tc_fence_after();
-          const bool skip = SKIP && skip_pv[t];
-          if (!skip) {
-            if (!v_ready) {
-              if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
-              tc_fence_after();
-              v_ready = true;
-            }
-            const uint64_t v0 = smem_desc_sw128(sV + st * L::kTile, BN * 128, 1024);
-            const uint32_t acc0 = pv_started[t];
-            const uint32_t d = tmem + 256 + t * 128, a = tmem + t * 128;
-            // keys [0, 64) as soon as their P is written, the rest after
-            if (leader) {
+          // Skip-softmax: the four softmax warps' votes for this tile were
+          // written before their P hand-off; a 32-key sub-tile is skipped when
+          // every row votes for it, and its P.V MMAs (two 16-key steps) are not
+          // issued.  The softmax warps take the skipped keys' p out of their
+          // row sums one tile later.
+          uint32_t skip_bits = 0, vis_bits = 0;
+          if constexpr (SKIP) {
 #pragma unroll
-              for (int kk = 0; kk < BN / 32; ++kk)
-                mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, kk > 0 ? 1u : acc0);
-            }
-            __syncwarp();
-            if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) continue;
-            tc_fence_after();
-            if (leader) {
-#pragma unroll
-              for (int kk = BN / 32; kk < BN / 16; ++kk)
-                mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, 1u);
-            }
-            pv_started[t] = 1;
-          } else if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) {
-            continue;
+            for (int u = 0; u < 4; ++u) vis_bits |= uint32_t(j * BN + 32 * u < g[t].k_end) << u;
+            skip_bits = and4_shared(votes + (t * 2 + (tile_c[t] & 1)) * 4) & vis_bits;
           }
+          if (!v_ready) {
+            if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
+            tc_fence_after();
+            v_ready = true;
+          }
+          const uint64_t v0 = smem_desc_sw128(sV + st * L::kTile, BN * 128, 1024);
+          uint32_t acc = pv_started[t];
+          const uint32_t d = tmem + 256 + t * 128, a = tmem + t * 128;
+          // keys [0, 64) as soon as their P is written, the rest after
+          if (leader) {
+#pragma unroll
+            for (int kk = 0; kk < BN / 32; ++kk) {
+              if ((skip_bits >> (kk / 2)) & 1u) continue;
+              mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, acc);
+              acc = 1u;
+            }
+          }
+          __syncwarp();
+          if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) continue;
+          tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int kk = BN / 32; kk < BN / 16; ++kk) {
+              if ((skip_bits >> (kk / 2)) & 1u) continue;
+              mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, acc);
+              acc = 1u;
+            }
+          }
+          pv_started[t] = __shfl_sync(0xffffffffu, acc, leader_lane);
           commit(&o_done[t]);
           ++tile_c[t];
           if (j + 1 < g[t].n) {
@@ -529,6 +557,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             issue_s(t, (c + 1) % kStages);
           }
+          // skip bookkeeping, after the MMAs are issued
+          if constexpr (SKIP) {
+            if (leader) {
+              n_vis += __popc(vis_bits);
+              n_skip += __popc(skip_bits);
+              if (p.skip_mask && skip_bits) {
+                for (int u = 0; u < 4; ++u) {
+                  if ((skip_bits >> u) & 1u) {
+                    const long long unit =
+                        (((long long)it.b * p.qb_max + it.r[t]) * p.h_q + it.hq[t]) * p.kt_max +
+                        (j * BN / 32 + u);
+                    atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
+                  }
+                }
+              }
+            }
+          }
         }
         if (ok) commit(&kv_empty[st]);
       }
@@ -538,6 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < kNQ; ++t) item_c[t] += g[t].n > 0 ? 1 : 0;
       kv_c += nmax;
       ++q_c;
+    }
+    if (SKIP && leader && p.skip_counts) {
+      atomicAdd(p.skip_counts + 0, n_vis);
+      atomicAdd(p.skip_counts + 1, n_skip);
     }
     // every MMA must be complete before the TMEM is released
 #pragma unroll
@@ -586,9 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_addr + t * 128;
     const uint32_t tO = tmem + lane_addr + 256 + t * 128;
     const float sl2 = p.scale_log2;
-    const int bar_id = 1 + t;
     uint32_t tile_c = 0;
-    unsigned long long n_vis = 0, n_skip = 0;
     bool alive = true;
 
     for (uint32_t n = 0; alive; ++n) {
@@ -608,22 +655,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       bool pv_any = false;
 
-      // One K/V tile of the dense (no skip) path.  From the second tile on,
-      // the exponentials of keys [0, 64) start at once against the current
-      // reference max while the tile max is taken alongside; only a row whose
-      // max grew past the lazy-rescale margin (after the first tile, rare)
-      // makes the warp redo them.  P of keys [0, 64) is handed to the MMA warp
-      // before the second half is computed, so the first half of P.V overlaps
-      // it.  The values written are those of computing the max first.
-      auto dense_step = [&](int j) -> bool {
+      // One K/V tile.  From the second tile on, the exponentials of keys
+      // [0, 64) start at once against the current reference max while the
+      // 32-key sub-tile maxima are taken alongside; a row whose max grew past
+      // the lazy-rescale margin (after the first tile, rare), or, with skip-
+      // softmax, a skipped sub-tile among those keys, makes the warp redo
+      // them.  P of keys [0, 64) is handed to the MMA warp before the second
+      // half is computed, so the first half of P.V overlaps it.  The values
+      // written are those of taking the maxima and decisions first.
+      // p summed per 32-key sub-tile over the row's last tile, and the
+      // correction once that tile's skip decisions are known: the skipped
+      // keys' p leave the row sum (their P.V MMAs were never issued)
+      float ps[4] = {0.f, 0.f, 0.f, 0.f}, ps_prev[4] = {0.f, 0.f, 0.f, 0.f};
+      // drop the skipped keys of the tile with warpgroup count c, local index
+      // jp, whose sub-tile sums are q, now worth `scale` each
+      auto drop_skipped = [&](uint32_t c, int jp, const float (&q)[4], float scale) {
+        alive = alive && __all_sync(0xffffffffu, wait_or_abort(&votes_ready[2 * t + (c & 1)], (c >> 1) & 1,
+                                                               abort_flag, p.err));
+        const uint32_t skip = and4_shared(votes + (t * 2 + (c & 1)) * 4);
+        float d = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (((skip >> u) & 1u) && jp * BN + 32 * u < g.k_end) d += q[u];
+        l -= d * scale;
+      };
+      auto step = [&](int j) -> bool {
         const bool ok =
             __all_sync(0xffffffffu, alive && wait_or_abort(&s_full[t], tile_c & 1, abort_flag, p.err));
         if (!ok) {
           alive = false;
           return false;
         }
-        tc_fence_after();
         uint32_t sr[4][32];
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
         tmem_wait_ld();
@@ -632,14 +696,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kbase = j * BN;
         if (kbase + BN > g.full_vis) mask_cols(sr, lim_row - kbase);
         float mref = (m_used == -INFINITY) ? 0.f : m_used;
-        float tmx;
-        uint64_t rs0 = 0;
+        float um[4];                                // raw maxima of the four 32-key sub-tiles
         const bool spec = j > 0;
         if (spec)
-          rs0 = exp64_to_tmem<true>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, tmx);
+          exp64_to_tmem<true>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, um, ps);
         else
-          tmx = max128(sr);
-        m_true = fmaxf(m_true, tmx * sl2);
+          max_sub4(sr, um);
+        if constexpr (SKIP) {
+          // vote per 32-key sub-tile: exp(sub-tile max - running max) <
+          // threshold; the MMA warp combines the four warps' votes
+          uint32_t my_votes = 0;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float t2 = um[u] * sl2;
+            const bool vote = !row_valid || (t2 == -INFINITY) || (t2 - m_true < p.thr_log2);
+            m_true = fmaxf(m_true, t2);
+            my_votes |= uint32_t(vote) << u;
+          }
+          const uint32_t wv = __reduce_and_sync(0xffffffffu, my_votes);
+          // the MMA warp reads it after the P hand-off below (which orders it);
+          // the warpgroup's own readers wait on votes_ready, arrived after it
+          if (lane == 0) votes[(t * 2 + (tile_c & 1)) * 4 + quad] = wv;
+        } else {
+          m_true = fmaxf(m_true, fmaxf(fmaxf(um[0], um[1]), fmaxf(um[2], um[3])) * sl2);
+        }
         // lazy rescale: move the reference max only when it grew by more than 2^8
         float alpha = 1.f;
         const bool grow = m_true > m_used + kRescaleLog2 || (m_used == -INFINITY && m_true > -INFINITY);
@@ -650,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!spec || __any_sync(0xffffffffu, grow)) {
           if (spec) tmem_wait_st();                 // the speculative half is overwritten
-          rs0 = exp64_to_tmem<false>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, tmx);
+          exp64_to_tmem<false>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, um, ps);
         }
         // rescale the O accumulator rows whose reference max moved
         if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -674,153 +754,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_half[t]);
-        float unused;
-        const uint64_t rs1 = exp64_to_tmem<false>(sr[2], sr[3], sr[2], sr[3], sl2, mref, tS + 32, unused);
-        float ra, rb;
-        f2_unpack(f2_add(rs0, rs1), ra, rb);
-        l = l * alpha + (ra + rb);
+        if (lane == 0) {
+          mbar_arrive(&p_half[t]);
+          if (SKIP) mbar_arrive(&votes_ready[2 * t + (tile_c & 1)]);
+        }
+        exp64_to_tmem<false>(sr[2], sr[3], sr[2], sr[3], sl2, mref, tS + 32, um, ps + 2);
+        l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[t]);
         ++tile_c;
         pv_any = true;
+        if constexpr (SKIP) {
+          // the previous tile's decisions are known by now
+          if (j > 0) drop_skipped(tile_c - 2, j - 1, ps_prev, alpha);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) ps_prev[u] = ps[u];
+        }
         return alive;
       };
 
-      for (int j = 0; j < g.n; ++j) {
-        if constexpr (!SKIP) {
-          if (!dense_step(j)) break;
-        } else {
-          // a failed wait anywhere turns the rest of the item into barrier-only
-          // iterations, so the warps never disagree about the named barrier below
-          bool ok = alive && wait_or_abort(&s_full[t], tile_c & 1, abort_flag, p.err);
-          ok = __all_sync(0xffffffffu, ok);
-          float s[128];
-          if (ok) {
-            tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tie(sr[c]);
-#pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] = -INFINITY;
-          }
-          const int kbase = j * BN;
-          if (kbase + BN > g.full_vis) {            // the tile holds masked entries for some row
-            const int lim = lim_row - kbase;
-#pragma unroll
-            for (int c = 0; c < 128; ++c)
-              if (c >= lim) s[c] = -INFINITY;
-          }
-
-          bool pv_skip = false;
-          // per 32-key sub-tile: vote skip when exp(tile max - running max) < threshold
-          uint32_t my_votes = 0;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float t2 = max32(s, u * 32) * sl2;
-            const bool vote = !row_valid || (t2 == -INFINITY) || (t2 - m_true < p.thr_log2);
-            m_true = fmaxf(m_true, t2);
-            my_votes |= uint32_t(vote) << u;
-          }
-          uint32_t wv = 0;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) wv |= uint32_t(__all_sync(0xffffffffu, (my_votes >> u) & 1u)) << u;
-          volatile uint32_t *vt = votes + (t * 2 + (j & 1)) * 4;
-          if (lane == 0) vt[quad] = wv | (ok ? 0u : 16u);
-          named_bar_sync(bar_id, 128);
-          const uint32_t v0 = vt[0], v1 = vt[1], v2 = vt[2], v3 = vt[3];
-          if ((v0 | v1 | v2 | v3) & 16u) {
-            alive = false;
-            continue;
-          }
-          uint32_t skip_bits = v0 & v1 & v2 & v3 & 15u;
-          uint32_t vis_bits = 0;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) vis_bits |= uint32_t(kbase + 32 * u < g.k_end) << u;
-          skip_bits &= vis_bits;
-          pv_skip = ((skip_bits | ~vis_bits) & 15u) == 15u;
-          if (quad == 0 && lane == 0) {
-            n_vis += __popc(vis_bits);
-            n_skip += __popc(skip_bits);
-            if (p.skip_mask && skip_bits) {
-              for (int u = 0; u < 4; ++u) {
-                if ((skip_bits >> u) & 1u) {
-                  const long long unit =
-                      (((long long)it.b * p.qb_max + it.r[t]) * p.h_q + hq) * p.kt_max + (kbase / 32 + u);
-                  atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
-                }
-              }
-            }
-            skip_pv[t] = pv_skip ? 1u : 0u;
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if ((skip_bits >> u) & 1u) {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) s[u * 32 + c] = -INFINITY;
-            }
-
-          // lazy rescale: move the reference max only when it grew by more than 2^8
-          float alpha = 1.f;
-          if (m_true > m_used + kRescaleLog2 || (m_used == -INFINITY && m_true > -INFINITY)) {
-            alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_true);
-            m_used = m_true;
-          }
-          const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-          // the same exponentials and row-sum order as the dense path, so a
-          // threshold that skips nothing reproduces it bit for bit
-          uint32_t sv[4][32];
-#pragma unroll
-          for (int c = 0; c < 128; ++c) sv[c >> 5][c & 31] = __float_as_uint(s[c]);
-          float unused;
-          const uint64_t rs0 = exp64_to_tmem<false>(sv[0], sv[1], sv[0], sv[1], sl2, mref, tS, unused);
-          const uint64_t rs1 = exp64_to_tmem<false>(sv[2], sv[3], sv[2], sv[3], sl2, mref, tS + 32, unused);
-          float ra, rb;
-          f2_unpack(f2_add(rs0, rs1), ra, rb);
-          l = l * alpha + (ra + rb);
-          tmem_wait_st();
-
-          // rescale the O accumulator rows whose reference max moved
-          if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
-            const bool okw =
-                __all_sync(0xffffffffu, wait_or_abort(&o_done[t], (tile_c - 1) & 1, abort_flag, p.err));
-            if (!okw) alive = false;
-            if (okw) {
-              tc_fence_after();
-#pragma unroll 1
-              for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + c * 32, o);
-                tmem_wait_ld();
-                tie(o);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                tmem_st32(tO + c * 32, o);
-              }
-              tmem_wait_st();
-            }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&p_half[t]);
-            mbar_arrive(&p_full[t]);
-          }
-          ++tile_c;
-          pv_any = pv_any || !pv_skip;
-        }
-      }
+      for (int j = 0; j < g.n; ++j)
+        if (!step(j)) break;
       if (!alive) break;
 
       // ---------------- epilogue ----------------
+      if (SKIP && g.n > 0) drop_skipped(tile_c - 1, g.n - 1, ps_prev, 1.f);
+      if (!alive) break;
       const bool have_o = g.n > 0;
       if (have_o) {
         alive = __all_sync(0xffffffffu, wait_or_abort(&o_done[t], (tile_c - 1) & 1, abort_flag, p.err));
@@ -861,10 +822,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (row_valid && p.lse)
         p.lse[(size_t)(sq.q0 + i) * p.h_q + hq] = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
-    }
-    if (SKIP && quad == 0 && lane == 0 && p.skip_counts) {
-      atomicAdd(p.skip_counts + 0, n_vis);
-      atomicAdd(p.skip_counts + 1, n_skip);
     }
   }
 
