@@ -214,6 +214,17 @@ ATTN_DEVICE uint32_t and4_shared(const volatile uint32_t *p) {
   return a & b & c & d;
 }
 
+// 16 columns of a warp's TMEM lanes from 16 consecutive registers.
+ATTN_DEVICE void tmem_st16(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+      : "memory");
+}
+
 // -inf for the columns at or beyond `lim` (keys the row may not see).
 ATTN_DEVICE void mask_cols(uint32_t (&sr)[4][32], int lim) {
 #pragma unroll
@@ -273,8 +284,9 @@ ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
     const int ac = (q < 16 ? 0 : 2) + (q & 1);
     acc[ac] = f2_add(acc[ac], f2_pack(p0, p1));
     pk[q] = pack_bf16x2(p0, p1);
+    if (q == 15) tmem_st16(taddr, pk);
   }
-  tmem_st32(taddr, pk);
+  tmem_st16(taddr + 16, pk + 16);
   if (MAX) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) um[u] = fmaxf(m[2 * u], m[2 * u + 1]);
