@@ -187,12 +187,13 @@ int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *
     return ATTN_E_CUDA;
   if (batch == 0) return ATTN_OK;
 
-  CUtensorMap qmap, kmap, vmap;
+  CUtensorMap qmap, kmap, vmap, omap;
   if (encode_3d(&qmap, q, d, h_q, total_q, kPrefillBlockM) ||
       encode_3d(&kmap, k, d, h_kv, total_k, kPrefillBlockN) ||
-      encode_3d(&vmap, v, d, h_kv, total_k, kPrefillBlockN))
+      encode_3d(&vmap, v, d, h_kv, total_k, kPrefillBlockN) ||
+      encode_3d(&omap, out, d, h_q, total_q, kPrefillBlockM))
     return ATTN_E_CUDA;
-  return launch_prefill(p, qmap, kmap, vmap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+  return launch_prefill(p, qmap, kmap, vmap, omap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
 }
 
 int attn_varlen_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,

@@ -246,6 +246,20 @@ ATTN_DEVICE void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *b
       : "memory");
 }
 
+// Tiled store shared -> global of one box of a 3-D tensor map (bulk async
+// group of the issuing thread; the source must stay untouched until
+// bulk_wait_read() returns).
+ATTN_DEVICE void tma_store_3d(const CUtensorMap *map, const void *smem_src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+ATTN_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's bulk stores have finished reading shared memory
+ATTN_DEVICE void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's bulk stores are complete
+ATTN_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Non-tensor bulk copy global -> shared of `bytes` (multiple of 16, both
 // addresses 16-byte aligned), completing as transaction bytes on `bar`.
 ATTN_DEVICE void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {

@@ -75,7 +75,10 @@ struct Smem {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kNQ * kTile;
   static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kBar = kV + kStages * kTile;
+  // output staging: per query tile, 64 columns x 128 rows of bf16 (one store box)
+  static constexpr int kStageBytes = BM * 64 * 2;
+  static constexpr int kStage = kV + kStages * kTile;
+  static constexpr int kBar = kStage + kNQ * kStageBytes;
   // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], o_free[NQ],
   // p_half[NQ], sched_full[SD], sched_empty[SD], votes_ready[NQ][2]
   static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ + 2 * kSchedDepth + 2 * kNQ;
@@ -84,6 +87,7 @@ struct Smem {
   static constexpr int kUsed = kMisc + 128;
   // at least ~116 KB so that a single CTA (and its 512 TMEM columns) owns an SM
   static constexpr int kBytes = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
+  static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 ATTN_DEVICE uint8_t *align1024(uint8_t *p) {
@@ -304,7 +308,8 @@ ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
 template <int D, bool SKIP>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, PrefillParams p) {
+                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                   PrefillParams p) {
   using L = Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = align1024(smem_raw);
@@ -379,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
+    tma_prefetch_desc(&omap);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -801,40 +807,84 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      uint16_t *orow = p.out + ((size_t)(sq.q0 + i) * p.h_q + hq) * D;
+      if (have_o && g.r0 + BM <= sq.s_q) {
+        // A full 128-row tile: normalised rows go, 64 columns at a time, to this
+        // warpgroup's staging buffer in the store box's 128-byte-swizzled
+        // layout, and one thread writes each box with a TMA store, so the
+        // warps move on to the next item instead of waiting on 256-byte
+        // scattered row stores.
+        uint8_t *stg = sm + L::kStage + t * L::kStageBytes;
+        const bool issuer = quad == 0 && lane == 0;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(tO + c * 32, o);
+        for (int hh = 0; hh < D / 64; ++hh) {
+          uint32_t o[2][32];
+          tmem_ld32(tO + hh * 64, o[0]);
+          tmem_ld32(tO + hh * 64 + 32, o[1]);
           tmem_wait_ld();
-          tie(o);
-          if (c == D / 32 - 1) {
-            // the accumulator is free for the next item once the last chunk is read
+          tie(o[0]);
+          tie(o[1]);
+          if (hh == D / 64 - 1) {
+            // the accumulator is free for the next item once the last columns are read
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[t]);
           }
-        } else {
+          if (issuer) bulk_wait_read();              // the previous box has left the buffer
+          named_bar_sync(1 + t, 128);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if (row_valid) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t *v = &o[c >> 2][(c & 3) * 8];
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-            dst[v] = w;
+            w.x = pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv);
+            *reinterpret_cast<uint4 *>(stg + sw128_offset((uint32_t)row, (uint32_t)c)) = w;
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1 + t, 128);
+          if (issuer) {
+            tma_store_3d(&omap, stg, hh * 64, hq, sq.q0 + g.r0);
+            bulk_commit();
+          }
+        }
+      } else {
+        uint16_t *orow = p.out + ((size_t)(sq.q0 + i) * p.h_q + hq) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (have_o) {
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+            tie(o);
+            if (c == D / 32 - 1) {
+              // the accumulator is free for the next item once the last chunk is read
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&o_free[t]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          if (row_valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+              dst[v] = w;
+            }
           }
         }
       }
       if (row_valid && p.lse)
         p.lse[(size_t)(sq.q0 + i) * p.h_q + hq] = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
     }
+    if (quad == 0 && lane == 0) bulk_wait_all();   // output boxes written before the CTA ends
   }
 
   tc_fence_before();
@@ -866,7 +916,7 @@ int num_sms() {
 
 template <int D, bool SKIP>
 cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
-                     const CUtensorMap &vmap, cudaStream_t stream) {
+                     const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t stream) {
   const int smem = Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, SKIP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -877,7 +927,7 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUte
   static std::atomic<unsigned int> next_slot{0};
   PrefillParams q = p;
   q.work_slot = (int)(next_slot.fetch_add(1u) % kWorkSlots);
-  prefill_kernel<D, SKIP><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, q);
+  prefill_kernel<D, SKIP><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, omap, q);
   return cudaGetLastError();
 }
 
@@ -905,14 +955,14 @@ cudaError_t launch_exp2_selftest(const float *x, float *y, int n, cudaStream_t s
 }
 
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
-                           const CUtensorMap &vmap, cudaStream_t stream) {
+                           const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t stream) {
   if (p.batch == 0 || p.qb_max == 0) return cudaSuccess;
   const bool skip = p.thr_log2 > -INFINITY;
   if (p.d == 128)
-    return skip ? launch_t<128, true>(p, qmap, kmap, vmap, stream)
-                : launch_t<128, false>(p, qmap, kmap, vmap, stream);
-  return skip ? launch_t<64, true>(p, qmap, kmap, vmap, stream)
-              : launch_t<64, false>(p, qmap, kmap, vmap, stream);
+    return skip ? launch_t<128, true>(p, qmap, kmap, vmap, omap, stream)
+                : launch_t<128, false>(p, qmap, kmap, vmap, omap, stream);
+  return skip ? launch_t<64, true>(p, qmap, kmap, vmap, omap, stream)
+              : launch_t<64, false>(p, qmap, kmap, vmap, omap, stream);
 }
 
 }  // namespace attn
