@@ -35,6 +35,7 @@ EXPORTS = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_varlen_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_F, _P, _P, _P]),
     "attn_varlen_fwd_ex": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_F, _F, _P, _P, _P, _P, _P]),
+    "attn_paged_prefill": (_I, [_P] * 6 + [_I] * 11 + [_F, _F, _P, _P, _P, _P, _P]),
     "attn_paged_decode_workspace_size": (_S, [_I, _I, _I]),
     "attn_paged_decode": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _S, _P]),
     "attn_paged_decode_ex": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _P, _P, _S, _P]),
@@ -141,6 +142,39 @@ def attn_varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_q, max_k, causal=Tr
         int(max_q), int(max_k), h_q, h_kv, d, int(bool(causal)), scale, float(skip_threshold),
         _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _stream(stream))
     _check("attn_varlen_fwd", rc)
+    return out, lse
+
+
+def attn_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, max_q, max_k,
+                       causal=True, scale=None, page_size=16, out=None, lse=None, skip_threshold=0.0,
+                       skip_mask=None, skip_counts=None, want_lse=True, stream=None):
+    """Varlen GQA forward with K/V in a paged cache. q [Tq, h_q, d]; caches
+    [pages, page_size, h_kv, d]; block_table int32 [B, max_pages];
+    cu_seqlens_q int32 [B + 1]; seq_lens_k int32 [B].  Returns (out, lse)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(seq_lens_k, "seq_lens_k", torch.int32, 1)
+    if k_cache.shape != v_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape")
+    total_q, h_q, d = q.shape
+    num_pages, ps, h_kv, _ = k_cache.shape
+    if ps != page_size:
+        raise ValueError(f"cache page dimension {ps} != page_size {page_size}")
+    batch = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((total_q, h_q), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib.attn_paged_prefill(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k),
+        batch, total_q, int(max_q), int(max_k), num_pages, block_table.shape[1], page_size, h_q, h_kv, d,
+        int(bool(causal)), scale, float(skip_threshold), _ptr(skip_mask), _ptr(skip_counts), _ptr(out),
+        _ptr(lse), _stream(stream))
+    _check("attn_paged_prefill", rc)
     return out, lse
 
 

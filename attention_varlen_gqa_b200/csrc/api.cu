@@ -196,6 +196,77 @@ int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *
   return launch_prefill(p, qmap, kmap, vmap, omap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
 }
 
+int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                       const int32_t *block_table, const int32_t *cu_seqlens_q, const int32_t *seq_lens_k,
+                       int batch, int total_q, int max_q, int max_k, int num_pages, int max_pages_per_seq,
+                       int page_size, int h_q, int h_kv, int d, int causal, float scale,
+                       float skip_threshold, uint32_t *skip_mask, unsigned long long *skip_counts,
+                       attn_bf16 *out, float *lse, attn_stream_t stream) {
+  if (batch < 0 || total_q < 0 || max_q < 0 || max_k < 0 || num_pages < 0 || max_pages_per_seq < 0)
+    return ATTN_E_SHAPE;
+  if (page_size != kPageSize) return ATTN_E_PAGE_SIZE;
+  if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
+  int rc = check_threshold(skip_threshold);
+  if (rc) return rc;
+  if (batch > 0 && (max_q <= 0 || total_q <= 0 || num_pages <= 0 || max_pages_per_seq <= 0))
+    return ATTN_E_SHAPE;
+  if (!q || !k_cache || !v_cache || !block_table || !cu_seqlens_q || !seq_lens_k || !out) return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return ATTN_E_ALIGN;
+  if ((long long)max_q > (1ll << 24) || (long long)max_k > (1ll << 24) ||
+      (long long)num_pages * page_size > (1ll << 30) || (long long)max_pages_per_seq * page_size > (1ll << 30))
+    return ATTN_E_TOO_LARGE;
+  unsigned int *err = nullptr;
+  rc = device_state(&err);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  PrefillParams p{};
+  p.cu_q = cu_seqlens_q;
+  p.out = out;
+  p.lse = lse;
+  p.skip_mask = skip_mask;
+  p.skip_counts = skip_counts;
+  p.batch = batch;
+  p.total_q = total_q;
+  p.max_q = max_q;
+  p.max_k = max_k;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.group = h_q / h_kv;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.qb_max = (max_q + kPrefillBlockM - 1) / kPrefillBlockM;
+  p.kt_max = (max_k + kSkipTile - 1) / kSkipTile;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.thr_log2 = thr_to_log2(skip_threshold);
+  p.err = err;
+  p.paged = 1;
+  p.num_pages = num_pages;
+  p.max_pages = max_pages_per_seq;
+  p.block_table = block_table;
+  p.seq_lens_k = seq_lens_k;
+
+  if (skip_mask) {
+    const size_t bits = (size_t)batch * p.qb_max * h_q * p.kt_max;
+    if (bits && cudaMemsetAsync(skip_mask, 0, align_up(bits, 32) / 8, st) != cudaSuccess)
+      return ATTN_E_CUDA;
+  }
+  if (skip_counts && cudaMemsetAsync(skip_counts, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    return ATTN_E_CUDA;
+  if (batch == 0) return ATTN_OK;
+
+  CUtensorMap qmap, kmap, vmap, omap;
+  const long long slots = (long long)num_pages * page_size;
+  if (encode_3d(&qmap, q, d, h_q, total_q, kPrefillBlockM) ||
+      encode_3d(&kmap, k_cache, d, h_kv, slots, kPageSize) ||
+      encode_3d(&vmap, v_cache, d, h_kv, slots, kPageSize) ||
+      encode_3d(&omap, out, d, h_q, total_q, kPrefillBlockM))
+    return ATTN_E_CUDA;
+  return launch_prefill(p, qmap, kmap, vmap, omap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+}
+
 int attn_varlen_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
                     const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                     int batch, int total_q, int total_k, int max_q, int max_k,

@@ -55,6 +55,11 @@ struct PrefillParams {
   float scale_log2, thr_log2;
   unsigned int *err;
   int work_slot;                // work-claim counter of this launch (set by launch_prefill)
+  // paged K/V (chunked prefill): keys and values of sequence b live in the
+  // pages block_table[b, :] of a [num_pages, 16, h_kv, d] cache, s_k =
+  // seq_lens_k[b]; cu_k / total_k are unused then
+  int paged, num_pages, max_pages;
+  const int32_t *block_table, *seq_lens_k;
 };
 
 cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream);

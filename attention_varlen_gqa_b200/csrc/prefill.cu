@@ -176,12 +176,18 @@ ATTN_DEVICE Seq seq_at(const PrefillParams &p, int b) {
   Seq s;
   s.q0 = __ldg(p.cu_q + b);
   const int q1 = __ldg(p.cu_q + b + 1);
-  s.k0 = __ldg(p.cu_k + b);
-  const int k1 = __ldg(p.cu_k + b + 1);
   s.s_q = q1 - s.q0;
-  s.s_k = k1 - s.k0;
-  s.bad = (s.q0 < 0) | (s.s_q < 0) | (q1 > p.total_q) | (s.s_q > p.max_q) | (s.k0 < 0) | (s.s_k < 0) |
-          (k1 > p.total_k) | (s.s_k > p.max_k);
+  s.bad = (s.q0 < 0) | (s.s_q < 0) | (q1 > p.total_q) | (s.s_q > p.max_q);
+  if (p.paged) {
+    s.k0 = 0;
+    s.s_k = __ldg(p.seq_lens_k + b);
+    s.bad |= (s.s_k < 0) | (s.s_k > p.max_k) | (s.s_k > p.max_pages * kPageSize);
+  } else {
+    s.k0 = __ldg(p.cu_k + b);
+    const int k1 = __ldg(p.cu_k + b + 1);
+    s.s_k = k1 - s.k0;
+    s.bad |= (s.k0 < 0) | (s.s_k < 0) | (k1 > p.total_k) | (s.s_k > p.max_k);
+  }
   return s;
 }
 
@@ -432,13 +438,38 @@ __global__ void __launch_bounds__(kThreads, 1)
               !(ok = wait_or_abort(&kv_empty[s], ((kv_c / kStages) - 1) & 1, abort_flag, p.err)))
             break;
           mbar_arrive_expect_tx(&k_full[s], BN * D * 2);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d_hint(sm + L::kK + s * L::kTile + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
-                             sq.k0 + j * BN, keep);
           mbar_arrive_expect_tx(&v_full[s], BN * D * 2);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d_hint(sm + L::kV + s * L::kTile + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
-                             sq.k0 + j * BN, keep);
+          if (!p.paged) {
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d_hint(sm + L::kK + s * L::kTile + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
+                               sq.k0 + j * BN, keep);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d_hint(sm + L::kV + s * L::kTile + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
+                               sq.k0 + j * BN, keep);
+          } else {
+            // one 16-token page per box; a page past the sequence (or a bad
+            // block-table entry, reported) is read at a row beyond the cache,
+            // which the copy fills with zeros
+            const int32_t *bt = p.block_table + (size_t)it.b * p.max_pages;
+            for (int pg = 0; pg < BN / kPageSize; ++pg) {
+              const int tok = j * BN + pg * kPageSize;
+              int page = p.num_pages;
+              if (tok < sq.s_k) {
+                page = __ldg(bt + tok / kPageSize);
+                if (page < 0 || page >= p.num_pages) {
+                  raise_error(p.err, ATTN_DEVERR_BLOCK_TABLE);
+                  page = p.num_pages;
+                }
+              }
+              const uint32_t off = s * L::kTile + pg * kPageSize * 128;
+              for (int h = 0; h < D / 64; ++h) {
+                tma_load_3d_hint(sm + L::kK + off + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
+                                 page * kPageSize, keep);
+                tma_load_3d_hint(sm + L::kV + off + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
+                                 page * kPageSize, keep);
+              }
+            }
+          }
         }
         ++q_c;
       }
@@ -539,6 +570,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
             tc_fence_after();
             v_ready = true;
+            if (p.paged && j == (sq.s_k - 1) / BN && (sq.s_k % kPageSize) != 0) {
+              // the sequence's last page holds slots past its end (whatever the
+              // cache has there); their p is 0, but 0 * NaN is not, so the V
+              // rows are zeroed before the P.V MMAs read them
+              const int r0 = sq.s_k - j * BN, r1 = (r0 + kPageSize - 1) / kPageSize * kPageSize;
+              for (int x = lane; x < (r1 - r0) * (D / 64) * 8; x += 32) {
+                const int h = x / ((r1 - r0) * 8), rem = x - h * (r1 - r0) * 8;
+                const int r = r0 + rem / 8, ch = rem % 8;
+                *reinterpret_cast<uint4 *>(sm + L::kV + st * L::kTile + h * BN * 128 + r * 128 + ch * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
           }
           const uint64_t v0 = smem_desc_sw128(sV + st * L::kTile, BN * 128, 1024);
           uint32_t acc = pv_started[t];

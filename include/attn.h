@@ -168,6 +168,51 @@ ATTN_API int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const at
                        attn_bf16 *out, float *lse, attn_stream_t stream);
 
 /*
+ * attn_paged_prefill -- varlen GQA attention forward whose keys and values
+ * live in a paged cache: chunked prefill, or several query tokens per
+ * sequence against the cache (NVIDIA/Model-Optimizer PR 1941, "Add split-k
+ * decode kernel for skip softmax", What does this PR do?, fifth bullet: the
+ * dedicated decode kernel takes one-token decode only, and prefill and
+ * multi-token decode over the paged cache stay on the general flash-attention
+ * kernel).  Sequence b has
+ * s_q = cu_seqlens_q[b+1] - cu_seqlens_q[b] query tokens, which are the last
+ * s_q positions of its s_k = seq_lens_k[b] cached tokens when causal
+ * (bottom-right alignment: query row i sees keys j <= i + s_k - s_q).
+ *
+ *   q              [total_q, h_q, d] bf16, packed like attn_varlen_fwd's
+ *   k_cache,
+ *   v_cache        [num_pages, page_size, h_kv, d] bf16; token t of sequence
+ *                  b lives in page block_table[b, t / page_size], slot
+ *                  t % page_size (the attn_paged_decode layout)
+ *   block_table    [batch, max_pages_per_seq] int32; entries beyond a
+ *                  sequence's last page are never read
+ *   cu_seqlens_q   [batch + 1] int32 prefix sums over total_q
+ *   seq_lens_k     [batch] int32, 0 <= seq_lens_k[b] <= min(max_k,
+ *                  max_pages_per_seq * page_size)
+ *   page_size      16
+ *   max_q, max_k   bounds of s_q and s_k (size the grid and the skip mask)
+ *   skip_threshold, skip_mask, skip_counts
+ *                  as attn_varlen_fwd_ex (same units and bit layout, with
+ *                  KT = ceil(max_k / skip_tile))
+ *   out            [total_q, h_q, d] bf16;  lse [total_q, h_q] float32 or NULL
+ *
+ * Cache slots past a sequence's end in its last page may hold anything (they
+ * are neither attended to nor multiplied into the output).  A block-table
+ * entry outside [0, num_pages) sets ATTN_DEVERR_BLOCK_TABLE and that page is
+ * read as zeros; a bad cu_seqlens_q or seq_lens_k entry sets
+ * ATTN_DEVERR_CU_SEQLENS and the sequence is not written.  Shares the
+ * work-claim counters of attn_varlen_fwd (64 concurrent calls per device).
+ */
+ATTN_API int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                       const int32_t *block_table, const int32_t *cu_seqlens_q,
+                       const int32_t *seq_lens_k, int batch, int total_q, int max_q, int max_k,
+                       int num_pages, int max_pages_per_seq, int page_size,
+                       int h_q, int h_kv, int d, int causal, float scale,
+                       float skip_threshold, uint32_t *skip_mask,
+                       unsigned long long *skip_counts,
+                       attn_bf16 *out, float *lse, attn_stream_t stream);
+
+/*
  * attn_paged_decode_workspace_size -- bytes of workspace attn_paged_decode
  * needs for this shape (a pure host query; 0 is never returned for
  * batch * h_q > 0).  The dense schedule keeps, per (sequence, q-head, split),

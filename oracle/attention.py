@@ -424,6 +424,35 @@ def paged_decode(q, k_cache, v_cache, block_table, seq_lens, h_q, h_kv, scale,
     return out, lse, rec
 
 
+def paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, h_q, h_kv, causal, scale,
+                  threshold=0.0, page_size=16, block_m=128, tile_n=32, forced_skip=None, rows=None):
+    """Varlen GQA attention forward whose keys and values live in a paged cache
+    (chunked prefill / multi-token decode against the cache).
+
+    NVIDIA/Model-Optimizer PR 1941 "Add split-k decode kernel for skip
+    softmax", What does this PR do?, fifth bullet: prefill and multi-token
+    decode over the paged cache are attention over the same cache with
+    several query tokens per sequence.  The result is that of
+    ``varlen_attention`` on the sequence's keys and values gathered from its
+    pages: sequence b has the queries cu_seqlens_q[b]:cu_seqlens_q[b+1] and
+    the s_k = seq_lens_k[b] cached tokens; causal masking is bottom-right
+    aligned (the queries are the last s_q positions of the context).
+    Returns (out, lse, SkipRecord) like ``varlen_attention``.
+    """
+    lens = [int(x) for x in seq_lens_k]
+    kf, vf = [], []
+    for b, L in enumerate(lens):
+        kf.append(gather_paged(k_cache, block_table[b], L, page_size))
+        vf.append(gather_paged(v_cache, block_table[b], L, page_size))
+    shape = (0,) + tuple(np.asarray(k_cache).shape[2:])
+    k = np.concatenate(kf) if sum(lens) else np.zeros(shape, dtype=np.asarray(k_cache).dtype)
+    v = np.concatenate(vf) if sum(lens) else np.zeros(shape, dtype=np.asarray(v_cache).dtype)
+    cu_k = np.zeros(len(lens) + 1, dtype=np.int64)
+    cu_k[1:] = np.cumsum(lens)
+    return varlen_attention(q, k, v, cu_seqlens_q, cu_k, h_q, h_kv, causal, scale, threshold=threshold,
+                            block_m=block_m, tile_n=tile_n, forced_skip=forced_skip, rows=rows)
+
+
 def split_partials(S, V, n_splits, tile):
     """Split-KV partial results for one row group (dense, no skipping).
 

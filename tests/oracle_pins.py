@@ -218,6 +218,48 @@ def pin_paged_equals_contiguous():
     assert np.all(out[3] == 0) and np.all(lse[3] == -math.inf)
 
 
+def pin_paged_prefill():
+    """Paged prefill == varlen forward on the test's own token-by-token gather
+    (causal, s_q < s_k, an empty sequence, a sequence with no queries), and
+    with one query per sequence == the decode oracle (two independent paths)."""
+    rng = np.random.default_rng(5)
+    page = 4
+    lens_k = np.array([9, 0, 13, 5])
+    lens_q = np.array([3, 0, 13, 0])
+    B, h_q, h_kv, d = len(lens_k), 4, 2, 8
+    pages_per = (lens_k + page - 1) // page
+    pool = int(pages_per.sum()) + 2
+    perm = rng.permutation(pool)
+    bt = np.zeros((B, int(pages_per.max())), dtype=np.int32)
+    off = 0
+    for b in range(B):
+        bt[b, :pages_per[b]] = perm[off:off + pages_per[b]]
+        off += pages_per[b]
+    kc = bf(rng.standard_normal((pool, page, h_kv, d)))
+    vc = bf(rng.standard_normal((pool, page, h_kv, d)))
+    q = bf(rng.standard_normal((int(lens_q.sum()), h_q, d)))
+    cu_q = cu_from_lens(lens_q)
+    out, lse, _ = oracle.paged_prefill(q, kc, vc, bt, cu_q, lens_k, h_q, h_kv, True, 0.5, page_size=page)
+    kcont, vcont = [], []
+    for b in range(B):
+        for t in range(lens_k[b]):
+            kcont.append(kc[bt[b, t // page], t % page])
+            vcont.append(vc[bt[b, t // page], t % page])
+    kcont = np.array(kcont).reshape(-1, h_kv, d)
+    vcont = np.array(vcont).reshape(-1, h_kv, d)
+    o2, l2, _ = oracle.varlen_attention(q, kcont, vcont, cu_q, cu_from_lens(lens_k), h_q, h_kv, True, 0.5)
+    close(out, o2)
+    close(lse, l2)
+    # one query per sequence, causal: the last position sees the whole context
+    q1 = bf(rng.standard_normal((B, h_q, d)))
+    o3, l3, _ = oracle.paged_prefill(q1, kc, vc, bt, np.arange(B + 1), lens_k, h_q, h_kv, True, 0.5,
+                                     page_size=page)
+    o4, l4, _ = oracle.paged_decode(q1, kc, vc, bt, lens_k, h_q, h_kv, 0.5, page_size=page)
+    close(o3, o4)
+    close(l3, l4)
+    assert np.all(o3[1] == 0) and np.all(l3[1] == -math.inf)
+
+
 def pin_split_combine():
     rng = np.random.default_rng(6)
     for n, splits, tile in ((1000, 32, 16), (37, 32, 4), (5, 8, 2), (300, 3, 128)):
@@ -446,7 +488,7 @@ def pin_decode_skip_matches_literal():
 
 ALL_PINS = [
     pin_bf16_codec, pin_two_by_two, pin_causal_two_by_two, pin_single_key, pin_uniform_scores,
-    pin_dense_matches_sdpa, pin_gqa_equals_repeated_mha, pin_paged_equals_contiguous,
+    pin_dense_matches_sdpa, pin_gqa_equals_repeated_mha, pin_paged_equals_contiguous, pin_paged_prefill,
     pin_split_combine, pin_peaked_decisions, pin_strict_threshold, pin_causal_dead_rows_vote_skip,
     pin_threshold_zero_is_dense, pin_threshold_one, pin_literal_equals_vectorised,
     pin_probabilities_sum_to_one, pin_smallseq_equals_varlen, pin_decode_skip_matches_literal,

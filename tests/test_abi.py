@@ -97,6 +97,31 @@ def test_varlen_argument_errors(A):
     assert varlen(A, mq=1 << 25, mk=1 << 25) == -13
 
 
+def paged_prefill(A, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cu=FAKE, sl=FAKE, batch=2, tq=64, mq=32, mk=64, pages=8, maxp=4,
+             ps=16, hq=8, hkv=2, d=128, causal=1, scale=0.1, thr=0.0, mask=None, counts=None, out=FAKE, lse=None,
+             stream=None)
+    a.update(kw)
+    return A.lib.attn_paged_prefill(a["q"], a["kc"], a["vc"], a["bt"], a["cu"], a["sl"], a["batch"], a["tq"],
+                                    a["mq"], a["mk"], a["pages"], a["maxp"], a["ps"], a["hq"], a["hkv"], a["d"],
+                                    a["causal"], a["scale"], a["thr"], a["mask"], a["counts"], a["out"],
+                                    a["lse"], a["stream"])
+
+
+def test_paged_prefill_argument_errors(A):
+    assert paged_prefill(A, ps=32) == -6
+    assert paged_prefill(A, hq=7) == -3
+    assert paged_prefill(A, d=96) == -4
+    assert paged_prefill(A, thr=1.5) == -5
+    assert paged_prefill(A, scale=0.0) == -10
+    assert paged_prefill(A, bt=None) == -1
+    assert paged_prefill(A, sl=None) == -1
+    assert paged_prefill(A, kc=FAKE + 8) == -2
+    assert paged_prefill(A, pages=0) == -8
+    assert paged_prefill(A, mq=0) == -8
+    assert paged_prefill(A, mq=1 << 25) == -13
+
+
 def decode(A, **kw):
     a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, batch=2, pages=4, maxp=2, ps=16, hq=8, hkv=2, d=128,
              thr=0.0, scale=0.1, mask=None, counts=None, out=FAKE, lse=None, ws=FAKE, wsb=1 << 30, stream=None)

@@ -35,6 +35,10 @@ MUTANTS = [
     ("paged_decode", "Kb[:, hk, :].T", "Kb[:, 0, :].T", "decode kv head ignored"),
     ("gather_paged", "cache[pages, t % page_size]", "cache[pages, t // page_size % page_size]",
      "page slot index"),
+    ("paged_prefill", "gather_paged(k_cache, block_table[b], L, page_size)",
+     "gather_paged(k_cache, block_table[0], L, page_size)", "paged prefill reads sequence 0's pages"),
+    ("paged_prefill", "cu_k, h_q, h_kv, causal, scale", "cu_k, h_q, h_kv, False, scale",
+     "paged prefill drops the causal mask"),
     ("combine_partials", "L = (w * ls).sum(axis=0)", "L = ls.sum(axis=0)", "combine drops weights"),
     ("combine_partials", "Msafe + np.log(", "np.log(", "combine LSE drops the max"),
     ("split_partials", "hi = min(n, (s + 1) * per * tile)", "hi = min(n, (s + 1) * per * tile - 1)",

@@ -139,6 +139,23 @@ def paged_decode(seq_lens, h_q=32, h_kv=8, d=128, page_size=16, seed=0, where="h
                 max_pages_per_seq=bt.shape[1], scale=1.0 / np.sqrt(d), values=where, seed=seed)
 
 
+def paged_prefill(lens_q, lens_k, h_q=8, h_kv=2, d=128, page_size=16, seed=0, where="host"):
+    """Packed queries [sum(lens_q), h_q, d] against a paged cache holding
+    lens_k[b] tokens per sequence (the block table a permutation of the pool);
+    the queries of a sequence are the last lens_q[b] positions of its context."""
+    rng = np.random.default_rng(seed)
+    lens_q = np.asarray(lens_q, dtype=np.int32)
+    lens_k = np.asarray(lens_k, dtype=np.int32)
+    bt, pool = paged_layout(lens_k, page_size, rng)
+    q = _values(rng, (int(lens_q.sum()), h_q, d), where, seed, 1)
+    kc = _values(rng, (max(pool, 1), page_size, h_kv, d), where, seed, 2)
+    vc = _values(rng, (max(pool, 1), page_size, h_kv, d), where, seed, 3)
+    return dict(q=q, k_cache=kc, v_cache=vc, block_table=bt, cu_seqlens_q=cu_from_lens(lens_q),
+                seq_lens_k=lens_k, lens_q=[int(x) for x in lens_q], lens_k=[int(x) for x in lens_k],
+                max_q=max(int(lens_q.max()), 1), max_k=max(int(lens_k.max()), 1), h_q=h_q, h_kv=h_kv, d=d,
+                page_size=page_size, num_pages=max(pool, 1), scale=1.0 / np.sqrt(d), values=where, seed=seed)
+
+
 def decode_lens(seed=0, batch=64, lo=1024, hi=32768):
     return [int(x) for x in np.random.default_rng(seed).integers(lo, hi + 1, batch)]
 
