@@ -348,12 +348,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // kSchedWarp, kSchedDepth items ahead), so CTAs that drew light items take
   // more of them; the claimed item numbers reach every role through a ring in
   // shared memory.  -1 ends the work.
-  auto pop_lane = [&](uint32_t n) -> int {      // single-thread roles
-    const uint32_t slot = n % kSchedDepth;
-    const int idx = wait_or_abort(&sched_full[slot], (n / kSchedDepth) & 1, abort_flag, p.err) ? ring[slot] : -1;
-    mbar_arrive(&sched_empty[slot]);
-    return idx;
-  };
   auto pop_warp = [&](uint32_t n) -> int {      // whole-warp roles
     const uint32_t slot = n % kSchedDepth;
     const bool okw =
@@ -404,76 +398,88 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsOther>();
   if (warp == kProducerWarp) {
     // =============== TMA producer ===============
-    if (lane == 0) {
+    // The whole warp runs the loop; lane 0 issues the Q copies and the
+    // contiguous K/V tiles.  With a paged cache a K/V tile is eight 16-token
+    // pages, and lanes 0-7 each read one page number and issue that page's
+    // boxes, so the many small copies do not queue behind one thread.
+    {
       const uint64_t keep = policy_evict_last();     // K/V tiles are re-read by other q-heads
       uint32_t kv_c = 0, q_c = 0;
       bool ok = true;
+      auto wait_all_p = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, p.err));
+      };
       for (uint32_t n = 0; ok; ++n) {
-        const int idx = pop_lane(n);
+        const int idx = pop_warp(n);
         if (idx < 0) break;
         const Item it = item_at(p, idx);
         const Seq sq = seq_at(p, it.b);
         if (sq.bad) continue;
         TileGeo g[kNQ];
         int nmax = 0;
+#pragma unroll
         for (int t = 0; t < kNQ; ++t) {
           g[t] = tile_geo(p, sq, it.r[t]);
           nmax = max(nmax, g[t].n);
         }
         if (nmax == 0) continue;
-        if (q_c > 0 && !(ok = wait_or_abort(q_empty, (q_c - 1) & 1, abort_flag, p.err))) break;
-        int qbytes = 0;
-        for (int t = 0; t < kNQ; ++t) qbytes += g[t].n > 0 ? BM * D * 2 : 0;
-        mbar_arrive_expect_tx(q_full, qbytes);
-        for (int t = 0; t < kNQ; ++t) {
-          if (g[t].n == 0) continue;
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sm + L::kQ + t * L::kTile + h * BM * 128, &qmap, q_full, h * 64, it.hq[t],
-                        sq.q0 + g[t].r0);
+        if (q_c > 0 && !(ok = wait_all_p(q_empty, (q_c - 1) & 1))) break;
+        if (lane == 0) {
+          int qbytes = 0;
+          for (int t = 0; t < kNQ; ++t) qbytes += g[t].n > 0 ? BM * D * 2 : 0;
+          mbar_arrive_expect_tx(q_full, qbytes);
+          for (int t = 0; t < kNQ; ++t) {
+            if (g[t].n == 0) continue;
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(sm + L::kQ + t * L::kTile + h * BM * 128, &qmap, q_full, h * 64, it.hq[t],
+                          sq.q0 + g[t].r0);
+          }
         }
         const int hk = it.hq[0] / p.group;
+        const int32_t *bt = p.paged ? p.block_table + (size_t)it.b * p.max_pages : nullptr;
         for (int j = 0; j < nmax; ++j, ++kv_c) {
           const int s = kv_c % kStages;
-          if (kv_c >= kStages &&
-              !(ok = wait_or_abort(&kv_empty[s], ((kv_c / kStages) - 1) & 1, abort_flag, p.err)))
-            break;
-          mbar_arrive_expect_tx(&k_full[s], BN * D * 2);
-          mbar_arrive_expect_tx(&v_full[s], BN * D * 2);
+          if (kv_c >= kStages && !(ok = wait_all_p(&kv_empty[s], ((kv_c / kStages) - 1) & 1))) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&k_full[s], BN * D * 2);
+            mbar_arrive_expect_tx(&v_full[s], BN * D * 2);
+          }
+          __syncwarp();
           if (!p.paged) {
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_3d_hint(sm + L::kK + s * L::kTile + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
-                               sq.k0 + j * BN, keep);
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_3d_hint(sm + L::kV + s * L::kTile + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
-                               sq.k0 + j * BN, keep);
-          } else {
+            if (lane == 0) {
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d_hint(sm + L::kK + s * L::kTile + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
+                                 sq.k0 + j * BN, keep);
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d_hint(sm + L::kV + s * L::kTile + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
+                                 sq.k0 + j * BN, keep);
+            }
+          } else if (lane < BN / kPageSize) {
             // one 16-token page per box; a page past the sequence (or a bad
             // block-table entry, reported) is read at a row beyond the cache,
             // which the copy fills with zeros
-            const int32_t *bt = p.block_table + (size_t)it.b * p.max_pages;
-            for (int pg = 0; pg < BN / kPageSize; ++pg) {
-              const int tok = j * BN + pg * kPageSize;
-              int page = p.num_pages;
-              if (tok < sq.s_k) {
-                page = __ldg(bt + tok / kPageSize);
-                if (page < 0 || page >= p.num_pages) {
-                  raise_error(p.err, ATTN_DEVERR_BLOCK_TABLE);
-                  page = p.num_pages;
-                }
-              }
-              const uint32_t off = s * L::kTile + pg * kPageSize * 128;
-              for (int h = 0; h < D / 64; ++h) {
-                tma_load_3d_hint(sm + L::kK + off + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
-                                 page * kPageSize, keep);
-                tma_load_3d_hint(sm + L::kV + off + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
-                                 page * kPageSize, keep);
+            const int tok = j * BN + lane * kPageSize;
+            int page = p.num_pages;
+            if (tok < sq.s_k) {
+              page = __ldg(bt + tok / kPageSize);
+              if (page < 0 || page >= p.num_pages) {
+                raise_error(p.err, ATTN_DEVERR_BLOCK_TABLE);
+                page = p.num_pages;
               }
             }
+            const uint32_t off = s * L::kTile + lane * kPageSize * 128;
+            for (int h = 0; h < D / 64; ++h) {
+              tma_load_3d_hint(sm + L::kK + off + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
+                               page * kPageSize, keep);
+              tma_load_3d_hint(sm + L::kV + off + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
+                               page * kPageSize, keep);
+            }
           }
+          __syncwarp();
         }
         ++q_c;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         // let copies still in flight land before the CTA's shared memory is released
         if (q_c > 0) drain(q_full, (q_c - 1) & 1);
         for (uint32_t x = kv_c > kStages ? kv_c - kStages : 0; x < kv_c; ++x) {

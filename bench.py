@@ -53,7 +53,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip"], default="all",
                     help="profiling aid: run a single operation (no JSON line)")
-    ap.add_argument("--no-skip", action="store_true", help="leave out the skip-softmax measurements")
+    ap.add_argument("--no-skip", action="store_true",
+                    help="leave out the skip-softmax and paged-prefill measurements")
     ap.add_argument("--no-cpu", action="store_true", help="leave out the CPU oracle baseline")
     ap.add_argument("--small", action="store_true",
                     help="profiling aid with --only: quarter-size decode / small-seq batches")
@@ -408,9 +409,10 @@ def main():
     agg = aggregate_ranks({"per": per, "total_ms": total_ms, "e2e_ms": e2e_ms_local, "flops": pre_flops,
                            "dec_bytes": dec_bytes, "ss_bytes": ss_bytes}, world, dev)
 
-    skip = None
+    skip = paged = None
     if not args.no_skip:
         skip = measure_skip(A, W, torch, dev, seed, pk, reps=3)
+        paged = measure_paged_prefill(A, W, torch, dev, seed, pk, reps=3)
 
     if rank != 0:
         if world > 1:
@@ -457,6 +459,7 @@ def main():
         "roofline": roofline,
         "rows": rows,
         "skip": skip,
+        "paged_prefill": paged,
         "cpu_baseline": cpu,
         "e2e": {"value": agg["e2e_value"], "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": agg["e2e_ms"],
@@ -530,6 +533,42 @@ def measure_skip(A, W, torch, dev, seed, pk, reps=3):
         res["decode"][str(thr)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
                                    "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"]}
     return res
+
+
+def measure_paged_prefill(A, W, torch, dev, seed, pk, reps=3):
+    """Chunked prefill against a paged cache: 16 sequences with contexts
+    U[2048, 16384] (seed), the last 512 positions as queries, h_q=32, h_kv=8,
+    d=128, 16-token pages, causal.  Not a step row: reported beside it."""
+    import numpy as np
+    rng = np.random.default_rng(1000 + seed)
+    lens_k = rng.integers(2048, 16385, 16)
+    lens_q = np.full(16, 512)
+    d = W.paged_prefill(lens_q, lens_k, h_q=32, h_kv=8, d=128, seed=seed, where="device")
+    bt = torch.from_numpy(d["block_table"]).to(dev)
+    cq = torch.from_numpy(d["cu_seqlens_q"]).to(dev)
+    sl = torch.from_numpy(d["seq_lens_k"]).to(dev)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(d["q"].shape[:2], dtype=torch.float32, device=dev)
+    pairs = sum(int(sq) * (int(sk) - int(sq)) + int(sq) * (int(sq) + 1) // 2 for sq, sk in zip(lens_q, lens_k))
+    flops = 4.0 * 128 * 32 * pairs
+
+    def run():
+        A.attn_paged_prefill(d["q"], d["k_cache"], d["v_cache"], bt, cq, sl, d["max_q"], d["max_k"],
+                             causal=True, out=out, lse=lse)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    return {"workload": "16 sequences, contexts U[2048,16384] (seed), last 512 positions as queries, "
+                        "h 32/8, d 128, page 16, causal",
+            "ms": ms, "flops": flops, "tflops": flops / ms / 1e9, "frac_of_measured": flops / ms / 1e9 / pk["bf16"],
+            "lens_k": [int(x) for x in lens_k]}
 
 
 if __name__ == "__main__":
