@@ -261,32 +261,20 @@ ATTN_DEVICE void max_sub4(const uint32_t (&sr)[4][32], float (&um)[4]) {
 }
 
 // p = 2^(s * sl2 - mref) for 64 columns of a row (32-column chunks a, b),
-// packed to bf16 pairs and stored to TMEM at `taddr` (32 columns); the sums
-// of p over chunk a and chunk b go to ps[0], ps[1].  With MAX, the raw maxima
-// of the four 32-column chunks a, b, c, d are taken alongside (on the ALU pipe
-// while the exponentials occupy MUFU) into um.
-template <bool MAX>
-ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
-                               const uint32_t (&c)[32], const uint32_t (&d)[32], float sl2, float mref,
-                               uint32_t taddr, float (&um)[4], float *ps) {
+// packed to bf16 pairs and stored to TMEM at `taddr` (32 columns, as two
+// 16-column stores so that the first is under way while the rest is
+// computed); the sums of p over chunk a and chunk b go to ps[0], ps[1].
+ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32], float sl2, float mref,
+                               uint32_t taddr, float *ps) {
   const uint64_t scale2 = f2_pack(sl2, sl2), neg_m2 = f2_pack(-mref, -mref);
   uint64_t acc[4];
-  float m[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = f2_pack(0.f, 0.f);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) m[k] = -INFINITY;
   uint32_t pk[32];
 #pragma unroll
   for (int q = 0; q < 32; ++q) {
     const int e = (2 * q) & 31;
     const uint32_t x0u = q < 16 ? a[e] : b[e], x1u = q < 16 ? a[e + 1] : b[e + 1];
-    if (MAX) {
-      // chains 0-1: a, 2-3: b, 4-5: c, 6-7: d
-      const int ch = (q < 16 ? 0 : 2) + (q & 1);
-      m[ch] = fmax3u(m[ch], x0u, x1u);
-      m[4 + ch] = fmax3u(m[4 + ch], q < 16 ? c[e] : d[e], q < 16 ? c[e + 1] : d[e + 1]);
-    }
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(x0u), __uint_as_float(x1u)), scale2, neg_m2);
     float x0, x1;
     f2_unpack(x, x0, x1);
@@ -297,10 +285,6 @@ ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
     if (q == 15) tmem_st16(taddr, pk);
   }
   tmem_st16(taddr + 16, pk + 16);
-  if (MAX) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) um[u] = fmaxf(m[2 * u], m[2 * u + 1]);
-  }
   float x0, x1;
   f2_unpack(f2_add(acc[0], acc[1]), x0, x1);
   ps[0] = x0 + x1;
@@ -724,14 +708,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       bool pv_any = false;
 
-      // One K/V tile.  From the second tile on, the exponentials of keys
-      // [0, 64) start at once against the current reference max while the
-      // 32-key sub-tile maxima are taken alongside; a row whose max grew past
-      // the lazy-rescale margin (after the first tile, rare), or, with skip-
-      // softmax, a skipped sub-tile among those keys, makes the warp redo
-      // them.  P of keys [0, 64) is handed to the MMA warp before the second
-      // half is computed, so the first half of P.V overlaps it.  The values
-      // written are those of taking the maxima and decisions first.
+      // One K/V tile: the four 32-key sub-tile maxima, the
+      // running max and lazy rescale (and the skip votes), then the
+      // exponentials in two halves; P of keys [0, 64) is handed to the MMA
+      // warp before the second half is computed, so the first half of P.V
+      // overlaps it.  (Starting the first half's exponentials before the
+      // maxima, with a redo when a row's max grew, measured 6 % slower: the
+      // maxima then trailed the exponentials on the path to the hand-off.)
       // p summed per 32-key sub-tile over the row's last tile, and the
       // correction once that tile's skip decisions are known: the skipped
       // keys' p leave the row sum (their P.V MMAs were never issued)
@@ -766,11 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kbase + BN > g.full_vis) mask_cols(sr, lim_row - kbase);
         float mref = (m_used == -INFINITY) ? 0.f : m_used;
         float um[4];                                // raw maxima of the four 32-key sub-tiles
-        const bool spec = j > 0;
-        if (spec)
-          exp64_to_tmem<true>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, um, ps);
-        else
-          max_sub4(sr, um);
+        max_sub4(sr, um);
         if constexpr (SKIP) {
           // vote per 32-key sub-tile: exp(sub-tile max - running max) <
           // threshold; the MMA warp combines the four warps' votes
@@ -797,10 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_true;
           mref = m_used;
         }
-        if (!spec || __any_sync(0xffffffffu, grow)) {
-          if (spec) tmem_wait_st();                 // the speculative half is overwritten
-          exp64_to_tmem<false>(sr[0], sr[1], sr[2], sr[3], sl2, mref, tS, um, ps);
-        }
+        exp64_to_tmem(sr[0], sr[1], sl2, mref, tS, ps);
         // rescale the O accumulator rows whose reference max moved
         if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
           const bool okw =
@@ -827,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&p_half[t]);
           if (SKIP) mbar_arrive(&votes_ready[2 * t + (tile_c & 1)]);
         }
-        exp64_to_tmem<false>(sr[2], sr[3], sr[2], sr[3], sl2, mref, tS + 32, um, ps + 2);
+        exp64_to_tmem(sr[2], sr[3], sl2, mref, tS + 32, ps + 2);
         l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
         tmem_wait_st();
         tc_fence_before();
