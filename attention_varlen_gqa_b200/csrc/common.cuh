@@ -141,6 +141,15 @@ ATTN_DEVICE void ldsm_x4_trans(uint32_t saddr, uint32_t &r0, uint32_t &r1, uint3
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(saddr));
 }
 
+// Transpose of an 8x8 b16 matrix held as one pair per lane (lane l: row l / 4,
+// columns 2 (l % 4) and 2 (l % 4) + 1, the lower column in the low half):
+// returns the same lane's pair of the transposed matrix.
+ATTN_DEVICE uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // warp reductions
 // ---------------------------------------------------------------------------

@@ -9,11 +9,12 @@
 //     32-token tiles, so every decision sees the running softmax maximum;
 //   * the threshold is a runtime argument.
 //
-// One CTA (4 warps) = one (sequence b, kv-head hk, split).  The G = h_q / h_kv
-// query heads of the group are the 16 rows (zero-padded) of a warp-level bf16
-// MMA, so a warp turns 16 tokens x 128 dims of K into the group's scores with
-// 16 m16n8k16 MMAs instead of thousands of scalar FMAs; this keeps the kernel
-// on the memory side of its roofline.  K and V pages are gathered through the
+// One CTA (4 warps) = one (sequence b, kv-head hk, split).  A warp turns 16
+// tokens x 128 dims of K into the group's scores with warp-level bf16 MMAs,
+// computed transposed (S^T = K Q^T, O^T = V^T P^T): the 16 tokens are the MMA
+// rows and the G = h_q / h_kv query heads of the group its columns, in tiles
+// of 8 (zero-padded), so a group of up to 8 heads costs 8 m16n8k16 MMAs per 16
+// tokens for the scores and 8 for P V.  K and V pages are gathered through the
 // block table with 3-D TMA copies (box = 64 dims x 1 head x 16 tokens,
 // 128-byte swizzle) into shared memory, 64 tokens (4 pages) per chunk, warp w
 // owning tokens [16w, 16w + 16) of every chunk.  Each warp keeps its own
@@ -48,6 +49,7 @@ constexpr int kDenseStages = 3;         // dense: K+V chunks in the ring
 constexpr int kSeqSlots = 5;            // sequential: chunk slots; a slot holds a chunk's K, then its V
 constexpr int kSeqLookahead = 2;        // sequential: PV pass lags the score pass
 constexpr int kSeqRing = kSeqLookahead + 1;
+constexpr int kRingFloats = 12;         // sequential: a lane's 8 scores + 4 head maxima per chunk
 static_assert(kSeqSlots > kSeqLookahead + 1, "K prefetch depth is kSeqSlots - kSeqLookahead");
 static_assert(kDecodeSplits == 32, "the combine kernel gives one lane per split");
 static_assert(kDecodeSplitTile % kChunk == 0, "a split is a whole number of chunks");
@@ -59,7 +61,7 @@ struct DecodeLayout {
   // dense: stage s holds K at 2s * kSlot and V at (2s + 1) * kSlot
   static constexpr int kK = 0;
   static constexpr int kS = SEQ ? kSeqSlots * kSlot : 2 * kDenseStages * kSlot;
-  static constexpr int kQmax = kS + (SEQ ? kSeqRing * kWarps * 32 * 10 * 4 : 0);   // 8 scores + 2 maxima
+  static constexpr int kQmax = kS + (SEQ ? kSeqRing * kWarps * 32 * kRingFloats * 4 : 0);
   static constexpr int kBar = kQmax + (SEQ ? 2 * kWarps * 16 * 4 : 0);
   static constexpr int kNumBars = SEQ ? 2 * kSeqSlots : kDenseStages;
   static constexpr int kBt = kBar + kNumBars * 8;                  // the CTA's block-table entries
@@ -82,62 +84,70 @@ ATTN_DEVICE uint32_t slot_addr(uint32_t slot, int tok, int c8) {
   return slot + (c8 >> 3) * (kChunk * 128) + tok * 128 + (((c8 & 7) ^ (tok & 7)) << 4);
 }
 
-// Per-lane geometry of the m16n8k16 fragments.
+// Per-lane geometry of the m16n8k16 fragments: g = the lane's row of an 8-row
+// fragment, cq = its first column of a column pair.
 struct Lane {
-  int w, lane, r0, r1, cq;
+  int w, lane, g, cq;
   ATTN_DEVICE explicit Lane(int tid)
-      : w(tid >> 5), lane(tid & 31), r0((tid & 31) >> 2), r1(((tid & 31) >> 2) + 8),
-        cq(((tid & 31) & 3) * 2) {}
+      : w(tid >> 5), lane(tid & 31), g((tid & 31) >> 2), cq(((tid & 31) & 3) * 2) {}
 };
 
-// Query fragments (A operand): rows = heads of the group, zero beyond G.
-template <int D>
-ATTN_DEVICE void load_q_frags(uint32_t (&qa)[D / 16][4], const uint16_t *qg, int G, const Lane &ln) {
+// Query fragments as the B operand of S^T = K Q^T: qb[n][kk] = the two 8-dim
+// halves of dims [16 kk, 16 kk + 16) of head 8 n + g (zero beyond G).
+template <int D, int NH>
+ATTN_DEVICE void load_q_frags(uint32_t (&qb)[NH][D / 16][2], const uint16_t *qg, int G, const Lane &ln) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const int d0 = kk * 16 + ln.cq;
-    qa[kk][0] = ln.r0 < G ? *reinterpret_cast<const uint32_t *>(qg + (size_t)ln.r0 * D + d0) : 0u;
-    qa[kk][1] = ln.r1 < G ? *reinterpret_cast<const uint32_t *>(qg + (size_t)ln.r1 * D + d0) : 0u;
-    qa[kk][2] = ln.r0 < G ? *reinterpret_cast<const uint32_t *>(qg + (size_t)ln.r0 * D + d0 + 8) : 0u;
-    qa[kk][3] = ln.r1 < G ? *reinterpret_cast<const uint32_t *>(qg + (size_t)ln.r1 * D + d0 + 8) : 0u;
+  for (int n = 0; n < NH; ++n) {
+    const int h = 8 * n + ln.g;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint16_t *src = qg + (size_t)h * D + kk * 16 + ln.cq;
+      qb[n][kk][0] = h < G ? *reinterpret_cast<const uint32_t *>(src) : 0u;
+      qb[n][kk][1] = h < G ? *reinterpret_cast<const uint32_t *>(src + 8) : 0u;
+    }
   }
 }
 
-// Scores of this warp's 16 tokens: sc[nt][e] = S(row e < 2 ? r0 : r1, token
-// 8 nt + cq + (e & 1)), scaled into the log2 domain, -inf for tokens at or
-// beyond L and for padding rows.  qm = per-row maxima over the 16 tokens.
-template <int D>
-ATTN_DEVICE void warp_scores(float (&sc)[2][4], float (&qm)[2], uint32_t kslot,
-                             const uint32_t (&qa)[D / 16][4], int tok_base, int L, int G, float sl2,
+// Scores of this warp's 16 tokens, computed transposed (M = the 16 tokens,
+// N = the group's heads in tiles of 8, K = head dims) so that a group of G <= 8
+// heads pads to 8 MMA columns, not 16 rows: sc[n][e] = S(head 8 n + cq + (e & 1),
+// token tok_base + g + 8 (e >> 1)) in the log2 domain, -inf for tokens at or
+// beyond L and for padding heads; qm[n][h] = max over the 16 tokens of head
+// 8 n + cq + h.
+template <int D, int NH>
+ATTN_DEVICE void warp_scores(float (&sc)[NH][4], float (&qm)[NH][2], uint32_t kslot,
+                             const uint32_t (&qb)[NH][D / 16][2], int tok_base, int L, int G, float sl2,
                              const Lane &ln) {
+  // even and odd k-steps accumulate separately: two chains of D / 32 MMAs
+  float acc[NH][2][4];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
+  for (int n = 0; n < NH; ++n)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-    const int tok = ln.w * 16 + nt * 8 + (ln.lane & 7);
+    for (int e = 0; e < 4; ++e) acc[n][0][e] = acc[n][1][e] = 0.f;
+  // A fragments (K rows): matrices (tokens 0-7, dims 0-7), (8-15, 0-7), (0-7, 8-15), (8-15, 8-15)
+  const int tok = ln.w * 16 + (ln.lane & 7) + ((ln.lane >> 3) & 1) * 8;
 #pragma unroll
-    for (int m = 0; m < D / 32; ++m) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(slot_addr(kslot, tok, m * 4 + (ln.lane >> 3)), b0, b1, b2, b3);
-      mma_bf16_16816(sc[nt], qa[2 * m], b0, b1);
-      mma_bf16_16816(sc[nt], qa[2 * m + 1], b2, b3);
-    }
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a[4];
+    ldsm_x4(slot_addr(kslot, tok, 2 * kk + (ln.lane >> 4)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int n = 0; n < NH; ++n) mma_bf16_16816(acc[n][kk & 1], a, qb[n][kk][0], qb[n][kk][1]);
   }
-  qm[0] = qm[1] = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int n = 0; n < NH; ++n) {
+    qm[n][0] = qm[n][1] = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int tok = tok_base + nt * 8 + ln.cq + (e & 1);
-      const int row = (e < 2) ? ln.r0 : ln.r1;
-      const float v = (tok < L && row < G) ? sc[nt][e] * sl2 : -INFINITY;
-      sc[nt][e] = v;
-      qm[e >> 1] = fmaxf(qm[e >> 1], v);
+      const int t = tok_base + ln.g + 8 * (e >> 1);
+      const int h = 8 * n + ln.cq + (e & 1);
+      const float v = (t < L && h < G) ? (acc[n][0][e] + acc[n][1][e]) * sl2 : -INFINITY;
+      sc[n][e] = v;
+      qm[n][e & 1] = fmaxf(qm[n][e & 1], v);
     }
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    qm[h] = fmaxf(qm[h], __shfl_xor_sync(0xffffffffu, qm[h], 1));
-    qm[h] = fmaxf(qm[h], __shfl_xor_sync(0xffffffffu, qm[h], 2));
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) qm[n][h] = fmaxf(qm[n][h], __shfl_xor_sync(0xffffffffu, qm[n][h], o));
   }
 }
 
@@ -157,79 +167,89 @@ ATTN_DEVICE void zero_tail_rows(uint8_t *base, uint32_t vslot, int tok_base, int
   __syncwarp();
 }
 
-// Online-softmax update of this warp's rows with its 16 tokens and O += P V.
-template <int D>
-ATTN_DEVICE void warp_pv(float (&o_acc)[D / 8][4], float (&m_w)[2], float (&l_w)[2],
-                         const float (&s)[2][4], const float (&qm)[2], uint32_t vslot, const Lane &ln) {
-  float alpha[2];
+// Online-softmax update of this warp's heads with its 16 tokens and
+// O^T += V^T P^T (M = head dims, N = heads, K = the 16 tokens).  The lane's
+// probabilities come out of the score fragment as (token g, heads cq, cq + 1)
+// pairs; one 8x8 register transpose per 8 tokens turns them into the B
+// fragment, which wants (tokens cq, cq + 1, head g).  o_acc[mt][n][e] = O(head
+// 8 n + cq + (e & 1), dim 16 mt + g + 8 (e >> 1)).
+template <int D, int NH>
+ATTN_DEVICE void warp_pv(float (&o_acc)[D / 16][NH][4], float (&m_w)[NH][2], float (&l_w)[NH][2],
+                         const float (&s)[NH][4], const float (&qm)[NH][2], uint32_t vslot, const Lane &ln) {
+  float alpha[NH][2];
+  bool rescale = false;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const float m_new = fmaxf(m_w[h], qm[h]);
-    alpha[h] = (m_w[h] == -INFINITY) ? 0.f : ex2(m_w[h] - m_new);
-    m_w[h] = m_new;
-    l_w[h] *= alpha[h];
-  }
-  if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+  for (int n = 0; n < NH; ++n)
 #pragma unroll
-    for (int t = 0; t < D / 8; ++t) {
-      o_acc[t][0] *= alpha[0];
-      o_acc[t][1] *= alpha[0];
-      o_acc[t][2] *= alpha[1];
-      o_acc[t][3] *= alpha[1];
+    for (int h = 0; h < 2; ++h) {
+      const float m_new = fmaxf(m_w[n][h], qm[n][h]);
+      alpha[n][h] = (m_w[n][h] == -INFINITY) ? 0.f : ex2(m_w[n][h] - m_new);
+      m_w[n][h] = m_new;
+      l_w[n][h] *= alpha[n][h];
+      rescale |= alpha[n][h] != 1.f;
     }
-  }
-  const float mr0 = (m_w[0] == -INFINITY) ? 0.f : m_w[0];
-  const float mr1 = (m_w[1] == -INFINITY) ? 0.f : m_w[1];
-  // A fragment (P): (rows r0, tokens 0-7), (rows r1, 0-7), (r0, 8-15), (r1, 8-15)
-  uint32_t pa[4];
+  if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const float p0 = ex2(s[nt][0] - mr0), p1 = ex2(s[nt][1] - mr0);
-    const float p2 = ex2(s[nt][2] - mr1), p3 = ex2(s[nt][3] - mr1);
-    l_w[0] += p0 + p1;
-    l_w[1] += p2 + p3;
-    pa[2 * nt + 0] = pack_bf16x2(p0, p1);
-    pa[2 * nt + 1] = pack_bf16x2(p2, p3);
-  }
-  const int mtx = ln.lane >> 3;
-  const int tok = ln.w * 16 + (mtx & 1) * 8 + (ln.lane & 7);
+    for (int t = 0; t < D / 16; ++t)
 #pragma unroll
-  for (int q2 = 0; q2 < D / 16; ++q2) {
-    // matrices: (tokens 0-7, dims 16 q2 + 0..7), (8-15, same), (0-7, + 8..15), (8-15, + 8..15)
-    uint32_t b0, b1, b2, b3;
-    ldsm_x4_trans(slot_addr(vslot, tok, 2 * q2 + (mtx >> 1)), b0, b1, b2, b3);
-    mma_bf16_16816(o_acc[2 * q2], pa, b0, b1);
-    mma_bf16_16816(o_acc[2 * q2 + 1], pa, b2, b3);
+      for (int n = 0; n < NH; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o_acc[t][n][e] *= alpha[n][e & 1];
+  }
+  uint32_t pb[NH][2];
+#pragma unroll
+  for (int n = 0; n < NH; ++n) {
+    const float mr0 = (m_w[n][0] == -INFINITY) ? 0.f : m_w[n][0];
+    const float mr1 = (m_w[n][1] == -INFINITY) ? 0.f : m_w[n][1];
+    const float p0 = ex2(s[n][0] - mr0), p1 = ex2(s[n][1] - mr1);   // token g
+    const float p2 = ex2(s[n][2] - mr0), p3 = ex2(s[n][3] - mr1);   // token g + 8
+    l_w[n][0] += p0 + p2;
+    l_w[n][1] += p1 + p3;
+    pb[n][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+    pb[n][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+  }
+  // A fragments (V^T) by transposing loads: matrices (tokens 0-7, dims 0-7),
+  // (0-7, 8-15), (8-15, 0-7), (8-15, 8-15) of the m-tile
+  const int tok = ln.w * 16 + (ln.lane & 7) + ((ln.lane >> 4) & 1) * 8;
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    uint32_t a[4];
+    ldsm_x4_trans(slot_addr(vslot, tok, 2 * mt + ((ln.lane >> 3) & 1)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int n = 0; n < NH; ++n) mma_bf16_16816(o_acc[mt][n], a, pb[n][0], pb[n][1]);
   }
 }
 
 // Merge the four warps' (m, l, O) and write the CTA's result: the split
 // partial (dense) or the normalised output and LSE (sequential).
-template <int D>
-ATTN_DEVICE void merge_and_store(uint8_t *merge_area, const float (&o_acc)[D / 8][4],
-                                 const float (&m_w)[2], float (&l_w)[2], bool dead, int G, int b,
+template <int D, int NH>
+ATTN_DEVICE void merge_and_store(uint8_t *merge_area, const float (&o_acc)[D / 16][NH][4],
+                                 const float (&m_w)[NH][2], float (&l_w)[NH][2], bool dead, int G, int b,
                                  int hk, int split, int nsplit, bool sequential, const DecodeParams &p,
                                  const Lane &ln) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    l_w[h] += __shfl_xor_sync(0xffffffffu, l_w[h], 1);
-    l_w[h] += __shfl_xor_sync(0xffffffffu, l_w[h], 2);
-  }
+  for (int n = 0; n < NH; ++n)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) l_w[n][h] += __shfl_xor_sync(0xffffffffu, l_w[n][h], o);
   float *mm = reinterpret_cast<float *>(merge_area);   // [warp][16]
   float *ll = mm + kWarps * 16;                         // [warp][16]
   float *oo = ll + kWarps * 16;                         // [warp][16][D]
-  if ((ln.lane & 3) == 0) {
-    mm[ln.w * 16 + ln.r0] = m_w[0];
-    mm[ln.w * 16 + ln.r1] = m_w[1];
-    ll[ln.w * 16 + ln.r0] = l_w[0];
-    ll[ln.w * 16 + ln.r1] = l_w[1];
-  }
 #pragma unroll
-  for (int t = 0; t < D / 8; ++t) {
-    *reinterpret_cast<float2 *>(oo + ((size_t)ln.w * 16 + ln.r0) * D + t * 8 + ln.cq) =
-        make_float2(o_acc[t][0], o_acc[t][1]);
-    *reinterpret_cast<float2 *>(oo + ((size_t)ln.w * 16 + ln.r1) * D + t * 8 + ln.cq) =
-        make_float2(o_acc[t][2], o_acc[t][3]);
+  for (int n = 0; n < NH; ++n) {
+    const int h = 8 * n + ln.cq;
+    if (ln.g == 0) {
+      mm[ln.w * 16 + h] = m_w[n][0];
+      mm[ln.w * 16 + h + 1] = m_w[n][1];
+      ll[ln.w * 16 + h] = l_w[n][0];
+      ll[ln.w * 16 + h + 1] = l_w[n][1];
+    }
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        oo[((size_t)ln.w * 16 + h + (e & 1)) * D + t * 16 + ln.g + 8 * (e >> 1)] = o_acc[t][n][e];
   }
   __syncthreads();
   for (int x = threadIdx.x; x < G * D; x += kThreads) {
@@ -282,7 +302,7 @@ ATTN_DEVICE void issue_pages(const CUtensorMap *map, uint8_t *slot, uint64_t *ba
   }
 }
 
-template <int D, bool SEQ>
+template <int D, bool SEQ, int NH>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           DecodeParams p) {
@@ -330,13 +350,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
   if (tid == 0 && (any_bad || bad_len))
     raise_error(p.err, any_bad ? ATTN_DEVERR_BLOCK_TABLE : ATTN_DEVERR_SEQ_LEN);
 
-  float o_acc[D / 8][4];
+  float o_acc[D / 16][NH][4];
+  float m_w[NH][2], l_w[NH][2];   // this warp's running max / this lane's partial sums, heads 8 n + cq + h
 #pragma unroll
-  for (int t = 0; t < D / 8; ++t)
+  for (int n = 0; n < NH; ++n) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o_acc[t][e] = 0.f;
-  float m_w[2] = {-INFINITY, -INFINITY};              // this warp's running max, rows r0 / r1
-  float l_w[2] = {0.f, 0.f};                          // partial row sums (this lane's columns)
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o_acc[t][n][e] = 0.f;
+    m_w[n][0] = m_w[n][1] = -INFINITY;
+    l_w[n][0] = l_w[n][1] = 0.f;
+  }
   bool failed = false;
 
   if (!any_bad && n > 0) {
@@ -346,8 +370,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       for (int s = 0; s < Lay::kNumBars; ++s) mbar_init(&bars[s], 1);
       fence_barrier_init();
     }
-    uint32_t qa[D / 16][4];
-    load_q_frags<D>(qa, p.q + ((size_t)b * p.h_q + (size_t)hk * G) * D, G, ln);
+    uint32_t qb[NH][D / 16][2];
+    load_q_frags<D, NH>(qb, p.q + ((size_t)b * p.h_q + (size_t)hk * G) * D, G, ln);
     __syncthreads();
     const float sl2 = p.scale_log2;
     unsigned long long n_vis = 0, n_skip = 0;
@@ -374,11 +398,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           const uint32_t kslot = sbase + Lay::kK + 2 * s * Lay::kSlot;
           const uint32_t vslot = kslot + Lay::kSlot;
           const int tok_base = (c0 + i) * kChunk + ln.w * 16;
-          float sc[2][4], qm[2];
-          warp_scores<D>(sc, qm, kslot, qa, tok_base, L, G, sl2, ln);
+          float sc[NH][4], qm[NH][2];
+          warp_scores<D, NH>(sc, qm, kslot, qb, tok_base, L, G, sl2, ln);
           if (tok_base < L) {
             zero_tail_rows<D>(base, vslot, tok_base, L, ln);
-            warp_pv<D>(o_acc, m_w, l_w, sc, qm, vslot, ln);
+            warp_pv<D, NH>(o_acc, m_w, l_w, sc, qm, vslot, ln);
           }
         }
         if (__syncthreads_or(!ok)) {
@@ -417,21 +441,27 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           const int sl = i % kSeqSlots;
           const bool ok = mbar_wait(&kfull[sl], (i / kSeqSlots) & 1, p.err) && !failed;
           const int tok_base = (c0 + i) * kChunk + ln.w * 16;
-          float sc[2][4], qm[2] = {-INFINITY, -INFINITY};
-          if (ok) warp_scores<D>(sc, qm, sbase + Lay::kK + sl * Lay::kSlot, qa, tok_base, L, G, sl2, ln);
+          float sc[NH][4], qm[NH][2];
+#pragma unroll
+          for (int nn = 0; nn < NH; ++nn) qm[nn][0] = qm[nn][1] = -INFINITY;
+          if (ok) warp_scores<D, NH>(sc, qm, sbase + Lay::kK + sl * Lay::kSlot, qb, tok_base, L, G, sl2, ln);
           float *qx = qmax + ((i & 1) * kWarps + ln.w) * 16;
-          if ((ln.lane & 3) == 0) {
-            qx[ln.r0] = qm[0];
-            qx[ln.r1] = qm[1];
+          if (ln.g == 0) {
+#pragma unroll
+            for (int nn = 0; nn < NH; ++nn) {
+              qx[8 * nn + ln.cq] = qm[nn][0];
+              qx[8 * nn + ln.cq + 1] = qm[nn][1];
+            }
           }
-          float *sr = s_ring + (((i % kSeqRing) * kWarps + ln.w) * 32 + ln.lane) * 10;
+          float *sr = s_ring + (((i % kSeqRing) * kWarps + ln.w) * 32 + ln.lane) * kRingFloats;
           if (ok) {
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nn = 0; nn < NH; ++nn) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) sr[nt * 4 + e] = sc[nt][e];
-            sr[8] = qm[0];
-            sr[9] = qm[1];
+              for (int e = 0; e < 4; ++e) sr[nn * 4 + e] = sc[nn][e];
+              sr[8 + 2 * nn] = qm[nn][0];
+              sr[9 + 2 * nn] = qm[nn][1];
+            }
           }
           if (__syncthreads_or(!ok)) {
             failed = true;
@@ -486,15 +516,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             if (okv) {
               const uint32_t vslot = sbase + Lay::kK + sl * Lay::kSlot;
               zero_tail_rows<D>(base, vslot, tok_base, L, ln);
-              const float *sr = s_ring + (((j % kSeqRing) * kWarps + ln.w) * 32 + ln.lane) * 10;
-              float sv[2][4], qm[2];
+              const float *sr = s_ring + (((j % kSeqRing) * kWarps + ln.w) * 32 + ln.lane) * kRingFloats;
+              float sv[NH][4], qm[NH][2];
 #pragma unroll
-              for (int nt = 0; nt < 2; ++nt)
+              for (int nn = 0; nn < NH; ++nn) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sv[nt][e] = sr[nt * 4 + e];
-              qm[0] = sr[8];
-              qm[1] = sr[9];
-              warp_pv<D>(o_acc, m_w, l_w, sv, qm, vslot, ln);
+                for (int e = 0; e < 4; ++e) sv[nn][e] = sr[nn * 4 + e];
+                qm[nn][0] = sr[8 + 2 * nn];
+                qm[nn][1] = sr[9 + 2 * nn];
+              }
+              warp_pv<D, NH>(o_acc, m_w, l_w, sv, qm, vslot, ln);
             }
           }
           // every warp is done with slot j % kSeqSlots: it takes the K of chunk j + kSeqSlots
@@ -524,7 +555,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     }
     __syncthreads();
   }
-  merge_and_store<D>(base + Lay::kK, o_acc, m_w, l_w, any_bad || failed, G, b, hk, split, nsplit, SEQ, p,
+  merge_and_store<D, NH>(base + Lay::kK, o_acc, m_w, l_w, any_bad || failed, G, b, hk, split, nsplit, SEQ, p,
                      ln);
 }
 
@@ -560,23 +591,30 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   if (p.lse && lane == 0) p.lse[row] = live ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
 }
 
-template <int D, bool SEQ>
+template <int D, bool SEQ, int NH>
 cudaError_t launch_k(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
   const size_t smem = DecodeLayout<D, SEQ>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, SEQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, SEQ, NH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(SEQ ? 1 : kDecodeSplits, p.h_kv, p.batch);
-  decode_kernel<D, SEQ><<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
+  decode_kernel<D, SEQ, NH><<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
   return cudaGetLastError();
+}
+
+// one n-tile of 8 heads for groups of up to 8 query heads, two up to 16
+template <int D, bool SEQ>
+cudaError_t launch_g(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                     cudaStream_t stream) {
+  return p.group <= 8 ? launch_k<D, SEQ, 1>(p, kmap, vmap, stream) : launch_k<D, SEQ, 2>(p, kmap, vmap, stream);
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
-  if (p.sequential) return launch_k<D, true>(p, kmap, vmap, stream);
-  cudaError_t e = launch_k<D, false>(p, kmap, vmap, stream);
+  if (p.sequential) return launch_g<D, true>(p, kmap, vmap, stream);
+  cudaError_t e = launch_g<D, false>(p, kmap, vmap, stream);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)p.batch * p.h_q;
   decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);

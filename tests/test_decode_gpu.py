@@ -89,7 +89,7 @@ LENS = [0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 1000, 4097, 5000]
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("heads", [(8, 2), (4, 4), (32, 8), (16, 1)])
+@pytest.mark.parametrize("heads", [(8, 2), (4, 4), (32, 8), (8, 1), (24, 2), (16, 1)])
 def test_dense_ragged(A, d, heads):
     h_q, h_kv = heads
     data = W.paged_decode(LENS, h_q=h_q, h_kv=h_kv, d=d, seed=h_q + d)
@@ -121,6 +121,15 @@ def test_skip_sets(A, thr):
     assert vis > 0
     if thr >= 0.1:
         assert skipped > 0
+
+
+@pytest.mark.parametrize("heads", [(8, 1), (24, 2), (16, 1)])
+def test_skip_sets_wide_groups(A, heads):
+    """Groups of 8, 12 and 16 query heads: one full, one partial and two full
+    8-head column tiles of the decode MMAs."""
+    data = _peaked([1, 33, 700, 3000], h_q=heads[0], h_kv=heads[1], seed=heads[0])
+    vis, _ = _check(A, data, 0.1)
+    assert vis > 0
 
 
 def test_skip_threshold_zero_is_dense(A):
