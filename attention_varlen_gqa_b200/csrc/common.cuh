@@ -278,17 +278,6 @@ ATTN_DEVICE void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uin
       : "memory");
 }
 
-// 16-byte asynchronous copy global -> shared (L2 only), and the arrive on an
-// mbarrier once all of this thread's earlier cp.async copies have landed (the
-// barrier's expected count must include this thread).
-ATTN_DEVICE void cp_async16(void *smem_dst, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
-               "l"(reinterpret_cast<uint64_t>(gsrc)) : "memory");
-}
-ATTN_DEVICE void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Same with an L2 eviction hint (cache policy from createpolicy).
 ATTN_DEVICE void tma_load_3d_hint(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
                                   int x, int y, int z, uint64_t policy) {

@@ -4,26 +4,55 @@
 // small-seq (s_q=1, s_kv<=16)") runs this case as three kernels (scores,
 // mask + softmax, output) with runtime dispatch over max_seqlen_kv in
 // {2,4,6,8,12,16}; the batch counts query tokens.  Here it is one fused,
-// memory-bound kernel.
+// memory-bound kernel: every byte of Q, K and V is read once.
 //
-// One warp per (query token, head) row, lane i holding dims [d/32 i,
-// d/32 (i + 1)) so every row load is one coalesced 256-byte transaction.  The
-// row's own key count picks the code path (up to 4, 8 or 16 keys), so no
-// work is spent on absent keys; all K and V loads of a row are issued before
-// the first use (128 registers a thread, 16 warps per SM: measured faster than
-// 24 or 32 warps with fewer loads in flight each).  The <= 16 partial dot products are reduced across
-// the warp by a reduce-scatter shuffle tree (16 shuffles for 16 keys instead
-// of 80); softmax, weights and O = P V stay in registers.  Measured against a
-// shared-memory ring fed by bulk or cp.async copies: 3.5 TB/s here vs 1.2-1.3
-// TB/s there (one 198 KB CTA per SM left too few warps for the compute).
+// A unit is (query token t, group of up to 16 heads).  Its bytes are the
+// group's query rows and, for each of the token's keys, the group's K and V
+// rows; with the heads in one group (h <= 16) a token's K (and V) rows of
+// all keys are one contiguous run of the packed [keys, heads, d] tensor.  One
+// persistent CTA per SM streams its units through a shared-memory byte ring:
+// a producer warp issues bulk asynchronous copies (one each for Q, K and V
+// of a token, or one per key when the heads span several groups) completing
+// on the unit's mbarrier, so the copies of the next units are in flight while
+// the current one is computed and no load waits in a register.  Sixteen
+// consumer warps take one head of the unit each: lane i holds dims [d/32 i,
+// d/32 (i + 1)) read from shared memory, the <= 16 partial dot products are
+// reduced across the warp by a reduce-scatter shuffle tree (16 shuffles for
+// 16 keys instead of 80), and softmax, weights and O = P V stay in registers.
+// The row's own key count picks the code path (up to 4, 8 or 16 keys).
+// Tokens are split between CTAs in equal shares of their bytes (2 + 2 s_kv
+// head rows a token) by a search over cu_seqlens_kv, so every CTA streams one
+// contiguous range of memory.
+#include <limits.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace attn {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
+constexpr int kHeads = 16;                       // heads per unit = consumer warps
+constexpr int kThreads = 32 * (kHeads + 1);      // + the producer warp
+constexpr int kDesc = 16;                        // units in flight (descriptor slots)
+constexpr uint32_t kRing = 224 * 1024;           // bytes of the unit ring
+constexpr int kProbe = 256;                      // probes per round of the partition search
+
+// n >= 0: key count; kBadRange / kTooLong: the row is written as zeros
+struct Unit {
+  int token, group, n, off;
+};
+constexpr int kBadRange = -1;
+constexpr int kTooLong = -2;
+
+struct Layout {
+  static constexpr uint32_t kDescOff = kRing;                        // [kDesc] Unit
+  static constexpr uint32_t kFull = kDescOff + kDesc * sizeof(Unit); // [kDesc] the unit's bytes landed
+  static constexpr uint32_t kEmpty = kFull + kDesc * 8;              // [kDesc] its consumers are done
+  static constexpr uint32_t kStart = kEmpty + kDesc * 8;             // [kDesc] ring position (producer)
+  static constexpr uint32_t kScratch = kStart + kDesc * 8;           // partition search
+  static constexpr size_t kBytes = kScratch + 16 + 128;              // + alignment slack
+};
+static_assert(Layout::kBytes <= 227 * 1024, "fits one CTA per SM");
 
 template <int D>
 struct LaneVec;
@@ -31,6 +60,11 @@ template <>
 struct LaneVec<128> {   // 4 bf16 per lane
   using T = uint2;
   static constexpr int E = 4;
+  static ATTN_DEVICE T lds(uint32_t a) {
+    T r;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+    return r;
+  }
   static ATTN_DEVICE void unpack(const T &x, float *f) {
     f[0] = bf16_lo(x.x); f[1] = bf16_hi(x.x); f[2] = bf16_lo(x.y); f[3] = bf16_hi(x.y);
   }
@@ -40,6 +74,11 @@ template <>
 struct LaneVec<64> {    // 2 bf16 per lane
   using T = uint32_t;
   static constexpr int E = 2;
+  static ATTN_DEVICE T lds(uint32_t a) {
+    T r;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(a));
+    return r;
+  }
   static ATTN_DEVICE void unpack(const T &x, float *f) { f[0] = bf16_lo(x); f[1] = bf16_hi(x); }
   static ATTN_DEVICE T pack(const float *f) { return pack_bf16x2(f[0], f[1]); }
 };
@@ -74,38 +113,22 @@ ATTN_DEVICE float reduce_scatter(float (&v)[NK], int lane) {
   return s;
 }
 
-ATTN_DEVICE uint2 ldg_stream(const uint2 *p) {
-  uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
-ATTN_DEVICE uint32_t ldg_stream(const uint32_t *p) {
-  uint32_t r;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
-}
-
-// One (query token, head) row with n <= NK keys.  V_WITH_K: issue the V
-// loads together with the K loads (more bytes in flight, more registers).
-template <int D, int NK, bool V_WITH_K>
-ATTN_DEVICE void row_attention(const SmallSeqParams &p, long long u, int hh, int k0, int n, int lane) {
+// One (query token, head) row with 0 < n <= NK keys, read from its unit in
+// shared memory: q at qa, key j's K row at ka + j * kstride, V row at
+// va + j * kstride (addresses already offset by this lane's dims).
+template <int D, int NK>
+ATTN_DEVICE void row_attention(const SmallSeqParams &p, uint32_t qa, uint32_t ka, uint32_t va,
+                               uint32_t kstride, int n, size_t row, int lane) {
   using LV = LaneVec<D>;
   using T = typename LV::T;
   constexpr int E = LV::E;
   static_assert(NK == 4 || NK == 8 || NK == 16, "power-of-two key counts for the reduce-scatter");
   constexpr int SH = (NK == 16) ? 1 : (NK == 8) ? 2 : 3;  // key of lane l after the reduce-scatter is l >> SH
-  const size_t stride = (size_t)p.h * D / E;           // one key in units of T
-  const T *kb = reinterpret_cast<const T *>(p.k + ((size_t)k0 * p.h + hh) * D) + lane;
-  const T *vb = reinterpret_cast<const T *>(p.v + ((size_t)k0 * p.h + hh) * D) + lane;
-  const T qv = ldg_stream(reinterpret_cast<const T *>(p.q + (size_t)u * D) + lane);
-  T kr[NK], vr[V_WITH_K ? NK : 1];
+  T kr[NK], vr[NK];
+  const T qv = LV::lds(qa);
 #pragma unroll
-  for (int j = 0; j < NK; ++j) {
-    if (j < n) {
-      kr[j] = ldg_stream(kb + j * stride);
-      if (V_WITH_K) vr[j] = ldg_stream(vb + j * stride);
-    }
-  }
+  for (int j = 0; j < NK; ++j)
+    if (j < n) kr[j] = LV::lds(ka + j * kstride);
   float q[E];
   LV::unpack(qv, q);
   float part[NK];
@@ -120,79 +143,232 @@ ATTN_DEVICE void row_attention(const SmallSeqParams &p, long long u, int hh, int
   }
   const int key = lane >> SH;
   const float sc = reduce_scatter<NK>(part, lane);
-  const float s2 = (key < n) ? sc * p.scale_log2 : -INFINITY;
-  const float m = warp_max(s2);
+  float m = (key < n) ? sc * p.scale_log2 : -INFINITY;
+  const float s2 = m;
+  // every key sits in 2^SH neighbouring lanes: the lane bits from SH up span each key once
+#pragma unroll
+  for (int o = 16; o >= (1 << SH); o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   const float pr = (key < n) ? ex2(s2 - m) : 0.f;
-  const float l = warp_sum(((lane & ((1 << SH) - 1)) == 0) ? pr : 0.f);
+  float l = pr;
+#pragma unroll
+  for (int o = 16; o >= (1 << SH); o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   const float inv = 1.f / l;
-  float o[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) o[e] = 0.f;
-  if (V_WITH_K) {
+  for (int j = 0; j < NK; ++j)
+    if (j < n) vr[j] = LV::lds(va + j * kstride);
+  float o_acc[E];
 #pragma unroll
-    for (int j = 0; j < NK; ++j) {
-      const float pj = __shfl_sync(0xffffffffu, pr, j << SH);
-      if (j < n) {
-        float vf[E];
-        LV::unpack(vr[j], vf);
+  for (int e = 0; e < E; ++e) o_acc[e] = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = fmaf(pj, vf[e], o[e]);
-      }
-    }
-  } else {
-    T vr2[NK];
+  for (int j = 0; j < NK; ++j) {
+    const float pj = __shfl_sync(0xffffffffu, pr, j << SH);
+    if (j < n) {
+      float vf[E];
+      LV::unpack(vr[j], vf);
 #pragma unroll
-    for (int j = 0; j < NK; ++j)
-      if (j < n) vr2[j] = ldg_stream(vb + j * stride);
-#pragma unroll
-    for (int j = 0; j < NK; ++j) {
-      const float pj = __shfl_sync(0xffffffffu, pr, j << SH);
-      if (j < n) {
-        float vf[E];
-        LV::unpack(vr2[j], vf);
-#pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = fmaf(pj, vf[e], o[e]);
-      }
+      for (int e = 0; e < E; ++e) o_acc[e] = fmaf(pj, vf[e], o_acc[e]);
     }
   }
 #pragma unroll
-  for (int e = 0; e < E; ++e) o[e] *= inv;
-  reinterpret_cast<T *>(p.out + (size_t)u * D)[lane] = LV::pack(o);
+  for (int e = 0; e < E; ++e) o_acc[e] *= inv;
+  reinterpret_cast<T *>(p.out + row * D)[lane] = LV::pack(o_acc);
   if (p.weights) {
     const float pt = __shfl_sync(0xffffffffu, pr, (lane < NK ? lane : 0) << SH);
-    if (lane < p.max_s_kv) p.weights[(size_t)u * p.max_s_kv + lane] = f32_to_bf16(lane < n ? pt * inv : 0.f);
+    if (lane < p.max_s_kv) p.weights[row * p.max_s_kv + lane] = f32_to_bf16(lane < n ? pt * inv : 0.f);
   }
 }
 
+// Token boundary of CTA c of G: the first t in [0, T] with t + cu[t] >= X_c,
+// X_c = c / G of T + cu[T] (so each CTA gets an equal share of the head rows
+// it must move, 2 + 2 s_kv a token); boundary 0 is 0 and boundary G is T.
+// Threads [0, kProbe) search this CTA's first boundary and [kProbe,
+// 2 kProbe) its last, each round probing kProbe evenly spaced tokens of the
+// current bracket.  For valid (non-decreasing) cu the result is exact; for
+// any cu, consecutive CTAs' ranges still cover [0, T), since boundary 0 is 0
+// and boundary G is T.
+ATTN_DEVICE void token_range(const SmallSeqParams &p, int *scratch, int &t0, int &t1) {
+  const int tid = threadIdx.x;
+  const int T = p.batch;
+  const int G = gridDim.x;
+  const int side = tid / kProbe;
+  const int pi = tid % kProbe;
+  const bool searcher = side < 2;
+  const int c = blockIdx.x + side;
+  int lo = 0, hi = T;            // the boundary lies in [lo, hi]; hi satisfies (or is T)
+  long long X = 0;
+  bool done = !searcher;
+  if (searcher) {
+    if (c == 0) {
+      hi = 0;
+      done = true;
+    } else if (c >= G) {
+      lo = T;
+      done = true;
+    } else {
+      const long long total = (long long)T + __ldg(p.cu + T);
+      X = total * c / G;
+    }
+  }
+  while (__syncthreads_or(!done)) {
+    if (tid < 2) scratch[tid] = INT_MAX;
+    __syncthreads();
+    const int span = hi - lo;
+    const int step = done ? 1 : (span + kProbe - 1) / kProbe;
+    const long long cand = lo + (long long)pi * step;
+    if (!done && cand < hi) {
+      const int t = (int)cand;
+      if ((long long)t + __ldg(p.cu + t) >= X) atomicMin(&scratch[side], pi);
+    }
+    __syncthreads();
+    if (!done) {
+      const int f = scratch[side];
+      if (f == INT_MAX) {
+        lo += ((span + step - 1) / step - 1) * step + 1;   // past the last probe
+      } else {
+        hi = lo + f * step;
+        lo = (f == 0) ? hi : lo + (f - 1) * step + 1;
+      }
+      done = lo >= hi;
+    }
+  }
+  if (pi == 0 && searcher) scratch[2 + side] = lo;
+  __syncthreads();
+  t0 = scratch[2];
+  t1 = scratch[3];
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 4) smallseq_kernel(SmallSeqParams p) {
-  using LV = LaneVec<D>;
-  const int lane = threadIdx.x & 31;
-  const long long units = (long long)p.batch * p.h;
-  const long long stride = (long long)gridDim.x * kWarps;
-  for (long long u = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5); u < units; u += stride) {
-    const int b = (int)(u / p.h);
-    const int hh = (int)(u - (long long)b * p.h);
-    const int k0 = __ldg(p.cu + b), k1 = __ldg(p.cu + b + 1);
-    const int n = k1 - k0;
-    const bool bad = (k0 < 0) | (n < 0) | (k1 > p.total_kv);
-    const bool too_long = !bad && n > p.max_s_kv;
-    if (bad | too_long | (n == 0)) {
+__global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  Unit *desc = reinterpret_cast<Unit *>(base + Layout::kDescOff);
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + Layout::kFull);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(base + Layout::kEmpty);
+  uint64_t *ustart = reinterpret_cast<uint64_t *>(base + Layout::kStart);
+  int *scratch = reinterpret_cast<int *>(base + Layout::kScratch);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.h;
+  const int ngroups = (H + kHeads - 1) / kHeads;
+  constexpr uint32_t kRow = D * 2;   // bytes of one head row
+
+  if (tid == 0) {
+    for (int s = 0; s < kDesc; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kHeads);
+    }
+    fence_barrier_init();
+  }
+  int t0, t1;
+  token_range(p, scratch, t0, t1);   // its barriers also publish the mbarrier init
+  const long long units = (long long)max(0, t1 - t0) * ngroups;
+
+  if (warp == kHeads) {
+    // ------------------------------ producer ------------------------------
+    // lane l holds cu[wb + l] and cu[wb + 32 + l]; lane 0 issues and keeps the ring
+    auto ld_cu = [&](int i) { return i <= p.batch ? __ldg(p.cu + i) : 0; };
+    int wb = t0;
+    int c_cur = ld_cu(wb + lane), c_nxt = ld_cu(wb + 32 + lane);
+    uint64_t hb = 0;            // ring bytes handed out so far
+    long long i = 0, o = 0;     // units issued / units known released
+    bool ok = true;
+    for (int t = t0; t < t1 && ok; ++t) {
+      if (t - wb == 32) {
+        wb += 32;
+        c_cur = c_nxt;
+        c_nxt = ld_cu(wb + 32 + lane);
+      }
+      const int j = t - wb;
+      const int k0 = __shfl_sync(0xffffffffu, c_cur, j);
+      const int k1 = __shfl_sync(0xffffffffu, j < 31 ? c_cur : c_nxt, (j + 1) & 31);
+      const int n = k1 - k0;
+      const bool bad = (k0 < 0) | (n < 0) | (k1 > p.total_kv);
+      const bool too_long = !bad && n > p.max_s_kv;
+      const int ncode = bad ? kBadRange : (too_long ? kTooLong : n);
       if (lane == 0) {
         if (bad) raise_error(p.err, ATTN_DEVERR_CU_SEQLENS);
         if (too_long) raise_error(p.err, ATTN_DEVERR_SMALLSEQ_LEN);
       }
-      float z[LV::E] = {};
-      reinterpret_cast<typename LV::T *>(p.out + (size_t)u * D)[lane] = LV::pack(z);
-      if (p.weights && lane < p.max_s_kv) p.weights[(size_t)u * p.max_s_kv + lane] = 0;
-      continue;
+      for (int g = 0; g < ngroups && ok; ++g) {
+        const int hg = min(kHeads, H - g * kHeads);
+        const uint32_t row = hg * kRow;
+        const uint32_t bytes = ncode > 0 ? row * (1 + 2 * n) : 0u;
+        uint64_t start = hb;
+        if (bytes != 0 && (hb % kRing) + bytes > kRing) start = hb + (kRing - hb % kRing);   // wrap
+        if (lane == 0) {
+          // release the oldest units until this one has a descriptor slot and room
+          while (o < i && (i - o >= kDesc || start + bytes - ustart[o % kDesc] > kRing)) {
+            if (!mbar_wait(&empty[o % kDesc], (uint32_t)(o / kDesc) & 1u, p.err)) {
+              ok = false;
+              break;
+            }
+            ++o;
+          }
+          if (ok) {
+            const int s = (int)(i % kDesc);
+            const uint32_t off = (uint32_t)(start % kRing);
+            desc[s] = Unit{t, g, ncode, (int)off};
+            ustart[s] = start;
+            mbar_arrive_expect_tx(&full[s], bytes);
+            if (bytes != 0) {
+              uint8_t *dst = base + off;
+              bulk_load(dst, p.q + ((size_t)t * H + g * kHeads) * D, row, &full[s]);
+              if (hg == H) {   // all heads in one group: the token's K (V) rows are one run
+                bulk_load(dst + row, p.k + (size_t)k0 * H * D, row * n, &full[s]);
+                bulk_load(dst + row * (1 + n), p.v + (size_t)k0 * H * D, row * n, &full[s]);
+              } else {
+                for (int jj = 0; jj < n; ++jj) {
+                  const size_t src = ((size_t)(k0 + jj) * H + g * kHeads) * D;
+                  bulk_load(dst + row * (1 + jj), p.k + src, row, &full[s]);
+                  bulk_load(dst + row * (1 + n + jj), p.v + src, row, &full[s]);
+                }
+              }
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        hb = start + bytes;
+        ++i;
+      }
     }
-    if (n <= 4)
-      row_attention<D, 4, true>(p, u, hh, k0, n, lane);
-    else if (n <= 8)
-      row_attention<D, 8, true>(p, u, hh, k0, n, lane);
-    else
-      row_attention<D, 16, true>(p, u, hh, k0, n, lane);
+    if (!ok && lane == 0) {
+      // let the copies still in flight land before the shared memory goes away
+      for (long long x = o; x < i; ++x) mbar_wait(&full[x % kDesc], (uint32_t)(x / kDesc) & 1u, nullptr);
+    }
+  } else {
+    // ------------------------------ consumers ------------------------------
+    const int w = warp;   // head of the unit's group
+    const uint32_t sbase = smem_u32(base);
+    using LV = LaneVec<D>;
+    for (long long i = 0; i < units; ++i) {
+      const int s = (int)(i % kDesc);
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(i / kDesc) & 1u, p.err))) break;
+      const Unit u = desc[s];
+      const int hg = min(kHeads, H - u.group * kHeads);
+      if (w < hg) {
+        const size_t row = (size_t)u.token * H + u.group * kHeads + w;
+        const int n = u.n;
+        if (n <= 0) {
+          float z[LV::E] = {};
+          reinterpret_cast<typename LV::T *>(p.out + row * D)[lane] = LV::pack(z);
+          if (p.weights && lane < p.max_s_kv) p.weights[row * p.max_s_kv + lane] = 0;
+        } else {
+          const uint32_t lo = lane * sizeof(typename LV::T);
+          const uint32_t qa = sbase + u.off + w * kRow + lo;
+          const uint32_t ka = sbase + u.off + hg * kRow + w * kRow + lo;
+          const uint32_t va = ka + n * hg * kRow;
+          const uint32_t ks = hg * kRow;
+          if (n <= 4)
+            row_attention<D, 4>(p, qa, ka, va, ks, n, row, lane);
+          else if (n <= 8)
+            row_attention<D, 8>(p, qa, ka, va, ks, n, row, lane);
+          else
+            row_attention<D, 16>(p, qa, ka, va, ks, n, row, lane);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
   }
 }
 
@@ -209,14 +385,11 @@ int num_sms() {
 
 template <int D>
 cudaError_t launch_d(const SmallSeqParams &p, cudaStream_t stream) {
-  int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smallseq_kernel<D>, kThreads, 0);
-  if (per_sm < 1) per_sm = 1;
-  const long long rows = (long long)p.batch * p.h;
-  const long long want = (rows + kWarps - 1) / kWarps;
-  const long long cap = (long long)num_sms() * per_sm;
-  const int grid = (int)(want < cap ? want : cap);
-  smallseq_kernel<D><<<grid, kThreads, 0, stream>>>(p);
+  cudaError_t e = cudaFuncSetAttribute(smallseq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Layout::kBytes);
+  if (e != cudaSuccess) return e;
+  const int grid = p.batch < num_sms() ? p.batch : num_sms();   // at least one token a CTA
+  smallseq_kernel<D><<<grid, kThreads, Layout::kBytes, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -88,3 +88,62 @@ def test_full_size_sampled(A):
     bsel = torch.as_tensor(bs, device="cuda")
     assert_close_bf16(out[bsel], ro)
     assert_close_bf16(wts[bsel], rw)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("h", [17, 40])
+def test_heads_in_several_groups(A, d, h):
+    """More than 16 heads: a token's rows travel as groups of 16 heads (the last
+    one partial), each key's rows of a group as their own copy."""
+    s = W.smallseq(seed=h + d, batch=300, h=h, d=d)
+    out, wts = _run(A, s, s["max_s_kv"])
+    ro, rw = oracle.smallseq_attention(s["q"], s["k"], s["v"], s["cu_seqlens_kv"], h, s["scale"], s["max_s_kv"])
+    assert_close_bf16(out, ro)
+    assert_close_bf16(wts, rw)
+    assert A.attn_get_last_device_error() == 0
+
+
+def test_bad_key_ranges_write_zeros(A):
+    """cu_seqlens_kv = [0, 4, 3, 22, 30, total + 3, total]: row 1 ends before
+    it starts, row 2 spans 19 keys (> max_s_kv), row 4 runs past the keys and
+    row 5 starts past them.  Those rows are zero, both error bits are raised,
+    rows 0 and 3 are exact."""
+    lens = np.array([4, 16, 2, 8, 6, 12], dtype=np.int32)
+    s = W.smallseq(seed=11, h=16, d=128, lens=lens)
+    total = int(s["cu_seqlens_kv"][-1])
+    cu_bad = s["cu_seqlens_kv"].copy()
+    cu_bad[2] = 3
+    cu_bad[5] = total + 3
+    q, k, v = (dev_bf16(s[n]) for n in ("q", "k", "v"))
+    out, wts = A.attn_smallseq_fwd(q, k, v, dev_i32(cu_bad), 16)
+    assert A.attn_get_last_device_error() == 1 | 8      # ATTN_DEVERR_CU_SEQLENS | ATTN_DEVERR_SMALLSEQ_LEN
+    for b in (1, 2, 4, 5):
+        assert torch.all(out[b] == 0) and torch.all(wts[b] == 0)
+    good = [0, 3]
+    ro, rw = oracle.smallseq_attention(s["q"], s["k"], s["v"], s["cu_seqlens_kv"], 16, s["scale"], 16,
+                                       batches=good)
+    assert_close_bf16(out, ro, where=np.s_[good])
+    assert_close_bf16(wts, rw, where=np.s_[good])
+
+
+@pytest.mark.parametrize("pattern", ["mostly_empty", "all_sixteen", "one_token"])
+def test_uneven_and_full_ring(A, pattern):
+    """Token ranges split by bytes when most rows are empty; back-to-back
+    16-key tokens (the largest units, the ring full); a batch of one."""
+    rng = np.random.default_rng(7)
+    if pattern == "mostly_empty":
+        lens = np.where(rng.random(5000) < 0.02, 16, 0).astype(np.int32)
+    elif pattern == "all_sixteen":
+        lens = np.full(3000, 16, dtype=np.int32)
+    else:
+        lens = np.array([9], dtype=np.int32)
+    s = W.smallseq(seed=8, h=16, d=128, lens=lens)
+    out, wts = _run(A, s, 16)
+    assert A.attn_get_last_device_error() == 0
+    pick = np.unique(np.concatenate([np.nonzero(lens)[0][:200], np.arange(min(50, len(lens)))]))
+    ro, rw = oracle.smallseq_attention(s["q"], s["k"], s["v"], s["cu_seqlens_kv"], 16, s["scale"], 16,
+                                       batches=pick)
+    assert_close_bf16(out, ro, where=np.s_[pick])
+    assert_close_bf16(wts, rw, where=np.s_[pick])
+    empty = torch.as_tensor(np.nonzero(lens == 0)[0], device="cuda")
+    assert torch.all(out[empty] == 0) and torch.all(wts[empty] == 0)
