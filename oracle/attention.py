@@ -537,3 +537,53 @@ def smallseq_attention(q, k, v, cu_seqlens_kv, h, scale, max_s_kv, batches=None)
             w[b, hh, 0, :] = 0.0
             w[b, hh, 0, :n] = P[0]
     return out, w
+
+
+def _as_f64(x):
+    """bf16 bit patterns (uint16) decoded exactly; any other array taken as values."""
+    x = np.asarray(x)
+    return bf16_bits_to_f64(x) if x.dtype == np.uint16 else x.astype(np.float64)
+
+
+def smallseq_backward(q, k, v, dout, weights, cu_seqlens_kv, h, scale, batches=None):
+    """Gradients of ``smallseq_attention`` from the attention weights it returned.
+
+    ROCm/TransformerEngine PR 461 "Integrate CK varlen cross attention for
+    small-seq (s_q=1, s_kv<=16)", description bullets: the backward runs as
+    grad_V, grad_attn, softmax backward and grad_Q / grad_K, and it reads the
+    attention weights the forward wrote into the reused auxiliary buffer
+    (forward write, backward read) rather than recomputing them.
+
+    For one (token b, head hh) with keys j = k0 .. k1-1 and P_j the saved
+    weight of key j, the steps in the page's order:
+      grad_V:       dV_j = P_j dO
+      grad_attn:    dP_j = <dO, v_j>
+      softmax bwd:  dS_j = P_j (dP_j - sum_i P_i dP_i)
+      grad_Q:       dQ   = scale * sum_j dS_j k_j
+      grad_K:       dK_j = scale * dS_j q
+    (the forward's scores are scale * <q, k_j>, so the chain rule puts the
+    scale on dQ and dK).  Rows with no key give dQ = 0.
+
+    q, dout: [B, h, d]; k, v: [total_kv, h, d]; weights: [B, h, 1, >= s_kv]
+    -- bf16 bit patterns (uint16) or float values.  Returns fp64 dq [B, h, d]
+    and dk, dv [total_kv, h, d]; rows and keys outside ``batches`` are NaN.
+    """
+    qf, kf, vf, of = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    wf = _as_f64(weights)
+    B, _, d = qf.shape
+    cu = np.asarray(cu_seqlens_kv, dtype=np.int64)
+    dq = np.full((B, h, d), np.nan)
+    dk = np.full(kf.shape, np.nan)
+    dv = np.full(vf.shape, np.nan)
+    for b in (range(B) if batches is None else batches):
+        k0, k1 = int(cu[b]), int(cu[b + 1])
+        n = k1 - k0
+        for hh in range(h):
+            P = wf[b, hh, 0, :n]                                  # [n] saved weights
+            dO = of[b, hh]                                        # [d]
+            dv[k0:k1, hh] = P[:, None] * dO[None, :]              # grad_V
+            dP = vf[k0:k1, hh] @ dO                               # grad_attn
+            dS = P * (dP - np.dot(P, dP))                         # softmax backward
+            dq[b, hh] = scale * (dS @ kf[k0:k1, hh]) if n else 0.0   # grad_Q
+            dk[k0:k1, hh] = scale * dS[:, None] * qf[b, hh][None, :]  # grad_K
+    return dq, dk, dv

@@ -486,10 +486,101 @@ def pin_decode_skip_matches_literal():
     assert n_skipped > 0
 
 
+
+# ---------------------------------------------------------------------------
+# small-seq backward
+# ---------------------------------------------------------------------------
+
+def _smallseq_case(seed, lens, h, d):
+    rng = np.random.default_rng(seed)
+    cu = cu_from_lens(np.asarray(lens))
+    B = len(lens)
+    q = rng.standard_normal((B, h, d))
+    k = rng.standard_normal((int(cu[-1]), h, d))
+    v = rng.standard_normal((int(cu[-1]), h, d))
+    do = rng.standard_normal((B, h, d))
+    return cu, q, k, v, do
+
+
+def pin_smallseq_backward_autograd():
+    """With the exact softmax as the saved weights, the backward equals torch
+    autograd (fp64) of L = sum dO . O through scores, softmax and P V."""
+    lens = [3, 16, 1, 8, 0, 5]
+    h, d, scale = 3, 8, 0.4
+    cu, q, k, v, do = _smallseq_case(13, lens, h, d)
+    B, max_s = len(lens), 16
+    W = np.zeros((B, h, 1, max_s))
+    dq_t, dk_t, dv_t = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        k0, k1 = int(cu[b]), int(cu[b + 1])
+        for hh in range(h):
+            qt = torch.tensor(q[b, hh], requires_grad=True)
+            kt = torch.tensor(k[k0:k1, hh], requires_grad=True)
+            vt = torch.tensor(v[k0:k1, hh], requires_grad=True)
+            P = torch.softmax(scale * (kt @ qt), dim=0)
+            (torch.tensor(do[b, hh]) * (P @ vt)).sum().backward()
+            W[b, hh, 0, :k1 - k0] = P.detach().numpy()
+            dq_t[b, hh] = qt.grad.numpy() if k1 > k0 else 0.0
+            dk_t[k0:k1, hh] = kt.grad.numpy()
+            dv_t[k0:k1, hh] = vt.grad.numpy()
+    dq, dk, dv = oracle.smallseq_backward(q, k, v, do, W, cu, h, scale)
+    close(dq, dq_t)
+    close(dk, dk_t)
+    close(dv, dv_t)
+    assert np.all(dq[4] == 0)
+
+
+def pin_smallseq_backward_finite_differences():
+    """Central differences of sum dO . O, with O from the oracle's own masked
+    softmax, match the backward in a few coordinates of q, k and v."""
+    lens = [4, 7]
+    h, d, scale, eps = 2, 6, 0.7, 1e-5
+    cu, q, k, v, do = _smallseq_case(14, lens, h, d)
+
+    def loss(q, k, v):
+        qq, kk, vv = q, k, v
+        tot = 0.0
+        for b in range(len(lens)):
+            k0, k1 = int(cu[b]), int(cu[b + 1])
+            for hh in range(h):
+                S = scale * (qq[b, hh][None, :] @ kk[k0:k1, hh].T)
+                O, _, _ = oracle.softmax_over_kept(S, np.ones_like(S, dtype=bool), vv[k0:k1, hh])
+                tot += float(do[b, hh] @ O[0])
+        return tot
+
+    W = np.zeros((len(lens), h, 1, 16))
+    for b in range(len(lens)):
+        k0, k1 = int(cu[b]), int(cu[b + 1])
+        for hh in range(h):
+            S = scale * (q[b, hh][None, :] @ k[k0:k1, hh].T)
+            W[b, hh, 0, :k1 - k0] = oracle.softmax_over_kept(S, np.ones_like(S, dtype=bool), v[k0:k1, hh])[2][0]
+    dq, dk, dv = oracle.smallseq_backward(q, k, v, do, W, cu, h, scale)
+    rng = np.random.default_rng(15)
+    for which, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(4):
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += eps
+            minus[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            fd = (loss(**{**args, which: plus}) - loss(**{**args, which: minus})) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), (which, idx, fd, grad[idx])
+
+
+def pin_smallseq_backward_single_key():
+    """One key: P = 1 whatever the score, so dQ = dK = 0 and dV = dO."""
+    cu, q, k, v, do = _smallseq_case(16, [1, 1], 2, 4)
+    W = np.ones((2, 2, 1, 1))
+    dq, dk, dv = oracle.smallseq_backward(bf(q), bf(k), bf(v), bf(do), W, cu, 2, 0.9)
+    close(dq, np.zeros_like(dq))
+    close(dk, np.zeros_like(dk))
+    close(dv, oracle.bf16_bits_to_f64(bf(do)))
+
 ALL_PINS = [
     pin_bf16_codec, pin_two_by_two, pin_causal_two_by_two, pin_single_key, pin_uniform_scores,
     pin_dense_matches_sdpa, pin_gqa_equals_repeated_mha, pin_paged_equals_contiguous, pin_paged_prefill,
     pin_split_combine, pin_peaked_decisions, pin_strict_threshold, pin_causal_dead_rows_vote_skip,
     pin_threshold_zero_is_dense, pin_threshold_one, pin_literal_equals_vectorised,
     pin_probabilities_sum_to_one, pin_smallseq_equals_varlen, pin_decode_skip_matches_literal,
+    pin_smallseq_backward_autograd, pin_smallseq_backward_finite_differences, pin_smallseq_backward_single_key,
 ]

@@ -45,6 +45,13 @@ MUTANTS = [
      "split drops a key"),
     ("smallseq_attention", "kf[k0:k1, hh, :]", "kf[k0:k1, 0, :]", "small-seq head ignored"),
     ("smallseq_attention", "w[b, hh, 0, :] = 0.0", "w[b, hh, 0, :] = 1.0", "weights padding"),
+    ("smallseq_backward", "dS = P * (dP - np.dot(P, dP))", "dS = P * dP", "softmax backward drops the row term"),
+    ("smallseq_backward", "dq[b, hh] = scale * (dS @ kf[k0:k1, hh])", "dq[b, hh] = (dS @ kf[k0:k1, hh])",
+     "grad_Q without the scale"),
+    ("smallseq_backward", "dP = vf[k0:k1, hh] @ dO", "dP = kf[k0:k1, hh] @ dO", "grad_attn reads K for V"),
+    ("smallseq_backward", "scale * dS[:, None] * qf[b, hh][None, :]", "scale * dS[:, None] * of[b, hh][None, :]",
+     "grad_K scales dO instead of q"),
+    ("smallseq_backward", "P[:, None] * dO[None, :]", "P[::-1, None] * dO[None, :]", "grad_V keys reversed"),
     ("literal_group_attention", "acc[r][c] *= alpha", "acc[r][c] *= 1.0", "missing O rescale"),
     ("literal_group_attention", "l[r] *= alpha", "l[r] *= 1.0", "missing l rescale"),
     ("bf16_bits_to_f64", "<< 16", "<< 15", "bf16 decode shift"),
