@@ -41,6 +41,7 @@ EXPORTS = {
     "attn_paged_decode_ex": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _P, _P, _S, _P]),
     "attn_paged_decode_static": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P]),
     "attn_smallseq_fwd": (_I, [_P] * 4 + [_I] * 5 + [_F, _P, _P, _P]),
+    "attn_smallseq_bwd": (_I, [_P] * 6 + [_I] * 5 + [_F, _P, _P, _P, _P]),
     "attn_get_last_device_error": (_I, [_P]),
     "attn_selftest_exp2": (_I, [_P, _P, _I, _P]),
 }
@@ -272,3 +273,30 @@ def attn_smallseq_fwd(q, k, v, cu_seqlens_kv, max_s_kv, scale=None, out=None, we
                                d, int(max_s_kv), scale, _ptr(out), _ptr(weights), _stream(stream))
     _check("attn_smallseq_fwd", rc)
     return out, weights
+
+
+def attn_smallseq_bwd(q, k, v, dout, weights, cu_seqlens_kv, max_s_kv=None, scale=None, dq=None, dk=None,
+                      dv=None, stream=None):
+    """Gradients of attn_smallseq_fwd from its attention weights [B, h, 1, max_s_kv].
+    dout [B, h, d].  Returns (dq [B, h, d], dk, dv [Tk, h, d])."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(dout, "dout", torch.bfloat16, 3)
+    _need(weights, "weights", torch.bfloat16, 4)
+    _need(cu_seqlens_kv, "cu_seqlens_kv", torch.int32, 1)
+    batch, h, d = q.shape
+    if max_s_kv is None:
+        max_s_kv = weights.shape[3]
+    if dq is None:
+        dq = torch.empty_like(q)
+    if dk is None:
+        dk = torch.empty_like(k)
+    if dv is None:
+        dv = torch.empty_like(v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib.attn_smallseq_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(weights), _ptr(cu_seqlens_kv),
+                               batch, k.shape[0], h, d, int(max_s_kv), scale, _ptr(dq), _ptr(dk), _ptr(dv),
+                               _stream(stream))
+    _check("attn_smallseq_bwd", rc)
+    return dq, dk, dv

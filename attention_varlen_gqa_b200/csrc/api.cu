@@ -457,6 +457,44 @@ int attn_smallseq_fwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v
   return launch_smallseq(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
 }
 
+int attn_smallseq_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v, const attn_bf16 *dout,
+                      const attn_bf16 *weights, const int32_t *cu_seqlens_kv, int batch, int total_kv,
+                      int h, int d, int max_s_kv, float scale, attn_bf16 *dq, attn_bf16 *dk,
+                      attn_bf16 *dv, attn_stream_t stream) {
+  if (batch < 0 || total_kv < 0) return ATTN_E_SHAPE;
+  if (h < 1) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (max_s_kv < 1 || max_s_kv > kSmallSeqMaxKv) return ATTN_E_SMALLSEQ;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
+  if (!q || !k || !v || !dout || !weights || !cu_seqlens_kv || !dq || !dk || !dv) return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return ATTN_E_ALIGN;
+  if (reinterpret_cast<uintptr_t>(weights) & 1u) return ATTN_E_ALIGN;
+  unsigned int *err = nullptr;
+  int rc = device_state(&err);
+  if (rc) return rc;
+  SmallSeqParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.cu = cu_seqlens_kv;
+  p.dout = dout;
+  p.weights_in = weights;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.batch = batch;
+  p.total_kv = total_kv;
+  p.h = h;
+  p.d = d;
+  p.max_s_kv = max_s_kv;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err;
+  return launch_smallseq_bwd(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+}
+
 int attn_selftest_exp2(const float *x, float *y, int n, attn_stream_t stream) {
   if (n < 0) return ATTN_E_SHAPE;
   if (n > 0 && (!x || !y)) return ATTN_E_NULL;

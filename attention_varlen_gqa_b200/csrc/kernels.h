@@ -21,9 +21,11 @@ constexpr int kMaxGroup = 16;         // largest h_q / h_kv supported by decode
 struct SmallSeqParams {
   const uint16_t *q, *k, *v;
   const int32_t *cu;
-  uint16_t *out, *weights;
+  uint16_t *out, *weights;             // forward outputs (weights may be null)
+  const uint16_t *dout, *weights_in;   // backward inputs: dO and the forward's weights
+  uint16_t *dq, *dk, *dv;              // backward outputs
   int batch, total_kv, h, d, max_s_kv;
-  float scale_log2;
+  float scale_log2, scale;
   unsigned int *err;
 };
 
@@ -63,6 +65,7 @@ struct PrefillParams {
 };
 
 cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream);
+cudaError_t launch_smallseq_bwd(const SmallSeqParams &p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float *x, float *y, int n, cudaStream_t stream);

@@ -37,9 +37,10 @@ constexpr int kDesc = 16;                        // units in flight (descriptor 
 constexpr uint32_t kRing = 224 * 1024;           // bytes of the unit ring
 constexpr int kProbe = 256;                      // probes per round of the partition search
 
-// n >= 0: key count; kBadRange / kTooLong: the row is written as zeros
+// n >= 0: key count; kBadRange / kTooLong: the row is written as zeros.
+// k0: the token's first key; off: the unit's byte offset in the ring.
 struct Unit {
-  int token, group, n, off;
+  int token, group, n, off, k0;
 };
 constexpr int kBadRange = -1;
 constexpr int kTooLong = -2;
@@ -178,15 +179,89 @@ ATTN_DEVICE void row_attention(const SmallSeqParams &p, uint32_t qa, uint32_t ka
   }
 }
 
-// Token boundary of CTA c of G: the first t in [0, T] with t + cu[t] >= X_c,
-// X_c = c / G of T + cu[T] (so each CTA gets an equal share of the head rows
-// it must move, 2 + 2 s_kv a token); boundary 0 is 0 and boundary G is T.
+// Backward of one (query token, head) row with 0 < n <= NK keys, from its
+// unit in shared memory (q at qa, dO at oa, key j's K and V rows at ka, va +
+// j * kstride) and the forward's weights (lane j < NK holds P_j).  The steps
+// of ROCm/TransformerEngine PR 461's backward:
+//   grad_attn     dP_j = <dO, v_j>            (reduce-scattered: lane l, key l >> SH)
+//   softmax bwd   dS_j = P_j (dP_j - sum_i P_i dP_i)
+//   grad_V        dV_j = P_j dO               (row j of dv)
+//   grad_K        dK_j = scale dS_j q         (row j of dk)
+//   grad_Q        dQ   = scale sum_j dS_j k_j
+// Key j's rows of this head start at element kv0 + j * kvs of dk and dv.
+template <int D, int NK>
+ATTN_DEVICE void row_backward(const SmallSeqParams &p, uint32_t qa, uint32_t oa, uint32_t ka, uint32_t va,
+                              uint32_t kstride, int n, float pw, size_t row, size_t kv0, size_t kvs,
+                              int lane) {
+  using LV = LaneVec<D>;
+  using T = typename LV::T;
+  constexpr int E = LV::E;
+  static_assert(NK == 4 || NK == 8 || NK == 16, "power-of-two key counts for the reduce-scatter");
+  constexpr int SH = (NK == 16) ? 1 : (NK == 8) ? 2 : 3;
+  float q[E], dO[E];
+  LV::unpack(LV::lds(qa), q);
+  LV::unpack(LV::lds(oa), dO);
+  T r[NK];
+#pragma unroll
+  for (int j = 0; j < NK; ++j)
+    if (j < n) r[j] = LV::lds(va + j * kstride);
+  float part[NK];
+#pragma unroll
+  for (int j = 0; j < NK; ++j) {
+    float vf[E];
+    LV::unpack(r[j], vf);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc = fmaf(dO[e], vf[e], acc);
+    part[j] = (j < n) ? acc : 0.f;
+  }
+  const int key = lane >> SH;
+  const float dp = reduce_scatter<NK>(part, lane);
+  const float pk = __shfl_sync(0xffffffffu, pw, key);
+  float t = (key < n) ? pk * dp : 0.f;
+#pragma unroll
+  for (int o = 16; o >= (1 << SH); o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  const float ds = (key < n) ? pk * (dp - t) : 0.f;
+#pragma unroll
+  for (int j = 0; j < NK; ++j)
+    if (j < n) r[j] = LV::lds(ka + j * kstride);
+  float dq[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) dq[e] = 0.f;
+#pragma unroll
+  for (int j = 0; j < NK; ++j) {
+    const float pj = __shfl_sync(0xffffffffu, pw, j);
+    const float dsj = __shfl_sync(0xffffffffu, ds, j << SH);
+    if (j < n) {
+      float a[E], kf[E];
+      const size_t at = kv0 + j * kvs;
+#pragma unroll
+      for (int e = 0; e < E; ++e) a[e] = pj * dO[e];
+      reinterpret_cast<T *>(p.dv + at)[lane] = LV::pack(a);
+      const float sk = p.scale * dsj;
+#pragma unroll
+      for (int e = 0; e < E; ++e) a[e] = sk * q[e];
+      reinterpret_cast<T *>(p.dk + at)[lane] = LV::pack(a);
+      LV::unpack(r[j], kf);
+#pragma unroll
+      for (int e = 0; e < E; ++e) dq[e] = fmaf(dsj, kf[e], dq[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) dq[e] *= p.scale;
+  reinterpret_cast<T *>(p.dq + row * D)[lane] = LV::pack(dq);
+}
+
+// Token boundary of CTA c of G: the first t in [0, T] with g(t) >= X_c, where
+// g(t) = wt t + wk cu[t] counts the head rows moved before token t (wt a
+// token, wk a key: 2 and 2 forward, 3 and 4 backward) and X_c = c / G of
+// g(T); boundary 0 is 0 and boundary G is T.
 // Threads [0, kProbe) search this CTA's first boundary and [kProbe,
 // 2 kProbe) its last, each round probing kProbe evenly spaced tokens of the
 // current bracket.  For valid (non-decreasing) cu the result is exact; for
 // any cu, consecutive CTAs' ranges still cover [0, T), since boundary 0 is 0
 // and boundary G is T.
-ATTN_DEVICE void token_range(const SmallSeqParams &p, int *scratch, int &t0, int &t1) {
+ATTN_DEVICE void token_range(const SmallSeqParams &p, int wt, int wk, int *scratch, int &t0, int &t1) {
   const int tid = threadIdx.x;
   const int T = p.batch;
   const int G = gridDim.x;
@@ -205,7 +280,7 @@ ATTN_DEVICE void token_range(const SmallSeqParams &p, int *scratch, int &t0, int
       lo = T;
       done = true;
     } else {
-      const long long total = (long long)T + __ldg(p.cu + T);
+      const long long total = (long long)wt * T + (long long)wk * __ldg(p.cu + T);
       X = total * c / G;
     }
   }
@@ -217,7 +292,7 @@ ATTN_DEVICE void token_range(const SmallSeqParams &p, int *scratch, int &t0, int
     const long long cand = lo + (long long)pi * step;
     if (!done && cand < hi) {
       const int t = (int)cand;
-      if ((long long)t + __ldg(p.cu + t) >= X) atomicMin(&scratch[side], pi);
+      if ((long long)wt * t + (long long)wk * __ldg(p.cu + t) >= X) atomicMin(&scratch[side], pi);
     }
     __syncthreads();
     if (!done) {
@@ -237,7 +312,8 @@ ATTN_DEVICE void token_range(const SmallSeqParams &p, int *scratch, int &t0, int
   t1 = scratch[3];
 }
 
-template <int D>
+// BWD: the backward (units carry q, dO, K, V; consumers run row_backward).
+template <int D, bool BWD>
 __global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -250,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p)
   const int H = p.h;
   const int ngroups = (H + kHeads - 1) / kHeads;
   constexpr uint32_t kRow = D * 2;   // bytes of one head row
+  constexpr uint32_t kQRows = BWD ? 2 : 1;   // query-side rows of a unit: q (and dO)
 
   if (tid == 0) {
     for (int s = 0; s < kDesc; ++s) {
@@ -259,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p)
     fence_barrier_init();
   }
   int t0, t1;
-  token_range(p, scratch, t0, t1);   // its barriers also publish the mbarrier init
+  token_range(p, BWD ? 3 : 2, BWD ? 4 : 2, scratch, t0, t1);   // its barriers also publish the mbarrier init
   const long long units = (long long)max(0, t1 - t0) * ngroups;
 
   if (warp == kHeads) {
@@ -291,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p)
       for (int g = 0; g < ngroups && ok; ++g) {
         const int hg = min(kHeads, H - g * kHeads);
         const uint32_t row = hg * kRow;
-        const uint32_t bytes = ncode > 0 ? row * (1 + 2 * n) : 0u;
+        const uint32_t bytes = ncode > 0 ? row * (kQRows + 2 * n) : 0u;
         uint64_t start = hb;
         if (bytes != 0 && (hb % kRing) + bytes > kRing) start = hb + (kRing - hb % kRing);   // wrap
         if (lane == 0) {
@@ -306,20 +383,23 @@ __global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p)
           if (ok) {
             const int s = (int)(i % kDesc);
             const uint32_t off = (uint32_t)(start % kRing);
-            desc[s] = Unit{t, g, ncode, (int)off};
+            desc[s] = Unit{t, g, ncode, (int)off, k0};
             ustart[s] = start;
             mbar_arrive_expect_tx(&full[s], bytes);
             if (bytes != 0) {
               uint8_t *dst = base + off;
-              bulk_load(dst, p.q + ((size_t)t * H + g * kHeads) * D, row, &full[s]);
+              const size_t qsrc = ((size_t)t * H + g * kHeads) * D;
+              bulk_load(dst, p.q + qsrc, row, &full[s]);
+              if (BWD) bulk_load(dst + row, p.dout + qsrc, row, &full[s]);
+              uint8_t *kd = dst + row * kQRows, *vd = kd + row * n;
               if (hg == H) {   // all heads in one group: the token's K (V) rows are one run
-                bulk_load(dst + row, p.k + (size_t)k0 * H * D, row * n, &full[s]);
-                bulk_load(dst + row * (1 + n), p.v + (size_t)k0 * H * D, row * n, &full[s]);
+                bulk_load(kd, p.k + (size_t)k0 * H * D, row * n, &full[s]);
+                bulk_load(vd, p.v + (size_t)k0 * H * D, row * n, &full[s]);
               } else {
                 for (int jj = 0; jj < n; ++jj) {
                   const size_t src = ((size_t)(k0 + jj) * H + g * kHeads) * D;
-                  bulk_load(dst + row * (1 + jj), p.k + src, row, &full[s]);
-                  bulk_load(dst + row * (1 + n + jj), p.v + src, row, &full[s]);
+                  bulk_load(kd + row * jj, p.k + src, row, &full[s]);
+                  bulk_load(vd + row * jj, p.v + src, row, &full[s]);
                 }
               }
             }
@@ -340,30 +420,58 @@ __global__ void __launch_bounds__(kThreads, 1) smallseq_kernel(SmallSeqParams p)
     const int w = warp;   // head of the unit's group
     const uint32_t sbase = smem_u32(base);
     using LV = LaneVec<D>;
+    // backward: lane j < max_s_kv holds P_j of this warp's head of unit i + 1,
+    // loaded one unit ahead (unit i is token t0 + i / ngroups, group i % ngroups)
+    auto load_weights = [&](long long i) -> float {
+      if (!BWD || i >= units || lane >= p.max_s_kv) return 0.f;
+      const long long t = t0 + i / ngroups;
+      const int hh = (int)(i % ngroups) * kHeads + w;
+      if (hh >= H) return 0.f;
+      return bf16_to_f32(__ldg(p.weights_in + ((size_t)t * H + hh) * p.max_s_kv + lane));
+    };
+    float pw_next = load_weights(0);
     for (long long i = 0; i < units; ++i) {
+      const float pw = pw_next;
+      pw_next = load_weights(i + 1);
       const int s = (int)(i % kDesc);
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(i / kDesc) & 1u, p.err))) break;
       const Unit u = desc[s];
       const int hg = min(kHeads, H - u.group * kHeads);
       if (w < hg) {
-        const size_t row = (size_t)u.token * H + u.group * kHeads + w;
+        const int hh = u.group * kHeads + w;
+        const size_t row = (size_t)u.token * H + hh;
         const int n = u.n;
+        float z[LV::E] = {};
         if (n <= 0) {
-          float z[LV::E] = {};
-          reinterpret_cast<typename LV::T *>(p.out + row * D)[lane] = LV::pack(z);
-          if (p.weights && lane < p.max_s_kv) p.weights[row * p.max_s_kv + lane] = 0;
+          if (BWD) {
+            reinterpret_cast<typename LV::T *>(p.dq + row * D)[lane] = LV::pack(z);
+          } else {
+            reinterpret_cast<typename LV::T *>(p.out + row * D)[lane] = LV::pack(z);
+            if (p.weights && lane < p.max_s_kv) p.weights[row * p.max_s_kv + lane] = 0;
+          }
         } else {
           const uint32_t lo = lane * sizeof(typename LV::T);
           const uint32_t qa = sbase + u.off + w * kRow + lo;
-          const uint32_t ka = sbase + u.off + hg * kRow + w * kRow + lo;
+          const uint32_t ka = sbase + u.off + kQRows * hg * kRow + w * kRow + lo;
           const uint32_t va = ka + n * hg * kRow;
           const uint32_t ks = hg * kRow;
-          if (n <= 4)
-            row_attention<D, 4>(p, qa, ka, va, ks, n, row, lane);
-          else if (n <= 8)
-            row_attention<D, 8>(p, qa, ka, va, ks, n, row, lane);
-          else
-            row_attention<D, 16>(p, qa, ka, va, ks, n, row, lane);
+          if (BWD) {
+            const uint32_t oa = qa + hg * kRow;
+            const size_t kv0 = ((size_t)u.k0 * H + hh) * D, kvs = (size_t)H * D;
+            if (n <= 4)
+              row_backward<D, 4>(p, qa, oa, ka, va, ks, n, pw, row, kv0, kvs, lane);
+            else if (n <= 8)
+              row_backward<D, 8>(p, qa, oa, ka, va, ks, n, pw, row, kv0, kvs, lane);
+            else
+              row_backward<D, 16>(p, qa, oa, ka, va, ks, n, pw, row, kv0, kvs, lane);
+          } else {
+            if (n <= 4)
+              row_attention<D, 4>(p, qa, ka, va, ks, n, row, lane);
+            else if (n <= 8)
+              row_attention<D, 8>(p, qa, ka, va, ks, n, row, lane);
+            else
+              row_attention<D, 16>(p, qa, ka, va, ks, n, row, lane);
+          }
         }
       }
       __syncwarp();
@@ -383,13 +491,13 @@ int num_sms() {
   return n;
 }
 
-template <int D>
+template <int D, bool BWD>
 cudaError_t launch_d(const SmallSeqParams &p, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(smallseq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(smallseq_kernel<D, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Layout::kBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.batch < num_sms() ? p.batch : num_sms();   // at least one token a CTA
-  smallseq_kernel<D><<<grid, kThreads, Layout::kBytes, stream>>>(p);
+  smallseq_kernel<D, BWD><<<grid, kThreads, Layout::kBytes, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -397,7 +505,12 @@ cudaError_t launch_d(const SmallSeqParams &p, cudaStream_t stream) {
 
 cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream) {
   if ((long long)p.batch * p.h == 0) return cudaSuccess;
-  return p.d == 128 ? launch_d<128>(p, stream) : launch_d<64>(p, stream);
+  return p.d == 128 ? launch_d<128, false>(p, stream) : launch_d<64, false>(p, stream);
+}
+
+cudaError_t launch_smallseq_bwd(const SmallSeqParams &p, cudaStream_t stream) {
+  if ((long long)p.batch * p.h == 0) return cudaSuccess;
+  return p.d == 128 ? launch_d<128, true>(p, stream) : launch_d<64, true>(p, stream);
 }
 
 }  // namespace attn

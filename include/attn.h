@@ -16,7 +16,8 @@
  *   attn_smallseq_fwd   s_q = 1, s_kv <= 16 cross attention over a huge batch,
  *                       also returning the attention weights
  *                       (ROCm/TransformerEngine PR 461, "Integrate CK varlen
- *                       cross attention for small-seq (s_q=1, s_kv<=16)").
+ *                       cross attention for small-seq (s_q=1, s_kv<=16)"),
+ *                       and attn_smallseq_bwd, its gradients from those weights.
  *
  * Skip-softmax (NVIDIA/TensorRT-LLM PR 9821, "Skip Softmax Attention"):
  * keys are visited in 32-key tiles in increasing order; a tile is skipped for
@@ -322,6 +323,36 @@ ATTN_API int attn_smallseq_fwd(const attn_bf16 *q, const attn_bf16 *k, const att
                       const int32_t *cu_seqlens_kv, int batch, int total_kv, int h, int d,
                       int max_s_kv, float scale, attn_bf16 *out, attn_bf16 *weights,
                       attn_stream_t stream);
+
+/*
+ * attn_smallseq_bwd -- gradients of attn_smallseq_fwd with respect to q, k
+ * and v, computed from the attention weights the forward returned
+ * (ROCm/TransformerEngine PR 461, description bullets: the backward's steps
+ * are grad_V, grad_attn, softmax backward and grad_Q / grad_K, and it reads
+ * the weights the forward wrote instead of recomputing them).  For token b,
+ * head hh, keys j of the token and P_j = weights[b, hh, 0, j]:
+ *   dV_j = P_j dO,  dP_j = <dO, v_j>,  dS_j = P_j (dP_j - sum_i P_i dP_i),
+ *   dQ = scale sum_j dS_j k_j,  dK_j = scale dS_j q.
+ *
+ *   q, k, v, cu_seqlens_kv, batch, total_kv, h, d, max_s_kv, scale
+ *                  as passed to attn_smallseq_fwd
+ *   dout           [batch, h, d] bf16: gradient of the loss w.r.t. `out`
+ *   weights        [batch, h, 1, max_s_kv] bf16, as attn_smallseq_fwd wrote it
+ *                  (required)
+ *   dq             [batch, h, d] bf16 output
+ *   dk, dv         [total_kv, h, d] bf16 outputs.  Every key inside a valid
+ *                  row's range is written once; keys outside every valid
+ *                  row's range (none when cu_seqlens_kv runs from 0 to
+ *                  total_kv) are left untouched.
+ * A row whose key range is invalid sets ATTN_DEVERR_CU_SEQLENS, a row with
+ * more than max_s_kv keys ATTN_DEVERR_SMALLSEQ_LEN; such a row's dq is zero
+ * and its keys' dk, dv are not written.  Empty rows give dq = 0.
+ */
+ATTN_API int attn_smallseq_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                               const attn_bf16 *dout, const attn_bf16 *weights,
+                               const int32_t *cu_seqlens_kv, int batch, int total_kv, int h, int d,
+                               int max_s_kv, float scale, attn_bf16 *dq, attn_bf16 *dk,
+                               attn_bf16 *dv, attn_stream_t stream);
 
 /*
  * attn_selftest_exp2 -- diagnostic: y[i] = the FMA-pipe approximation of 2^x[i]

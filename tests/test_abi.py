@@ -162,3 +162,25 @@ def test_smallseq_argument_errors(A):
     assert smallseq(A, cu=None) == -1
     assert smallseq(A, w=FAKE + 1) == -2
     assert smallseq(A, scale=-math.inf) == -10
+
+
+def smallseq_bwd(A, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, do=FAKE, w=FAKE, cu=FAKE, batch=3, tk=9, h=2, d=128, maxs=4, scale=0.1,
+             dq=FAKE, dk=FAKE, dv=FAKE, stream=None)
+    a.update(kw)
+    return A.lib.attn_smallseq_bwd(a["q"], a["k"], a["v"], a["do"], a["w"], a["cu"], a["batch"], a["tk"], a["h"],
+                                   a["d"], a["maxs"], a["scale"], a["dq"], a["dk"], a["dv"], a["stream"])
+
+
+def test_smallseq_bwd_argument_errors(A):
+    assert smallseq_bwd(A, maxs=0) == -7
+    assert smallseq_bwd(A, maxs=17) == -7
+    assert smallseq_bwd(A, d=32) == -4
+    assert smallseq_bwd(A, h=0) == -3
+    assert smallseq_bwd(A, batch=-1) == -8
+    assert smallseq_bwd(A, w=None) == -1
+    assert smallseq_bwd(A, do=None) == -1
+    assert smallseq_bwd(A, dk=None) == -1
+    assert smallseq_bwd(A, w=FAKE + 1) == -2
+    assert smallseq_bwd(A, dq=FAKE + 8) == -2
+    assert smallseq_bwd(A, scale=0.0) == -10

@@ -303,3 +303,30 @@ def smallseq(seed=0, batch=30720, h=16, d=128, choices=SMALLSEQ_BUCKETS, where="
     return dict(q=q, k=k, v=v, cu_seqlens_kv=cu, lens=lens, batch=batch, h=h, d=d,
                 max_s_kv=int(lens.max()) if batch else 1, scale=1.0 / np.sqrt(d),
                 values=where, seed=seed)
+
+
+def smallseq_grad_inputs(s, seed=0, where="host"):
+    """Backward inputs for a small-seq case ``s``: dO [B, h, d] ~ N(0, 1) and
+    saved weights [B, h, 1, max_s_kv] standing in for a forward's: per row,
+    uniform(0.05, 1) draws over the row's own keys scaled to sum to 1, zero
+    beyond; both bf16."""
+    B, h, d, ms = s["batch"], s["h"], s["d"], s["max_s_kv"]
+    lens = np.asarray(s["lens"])
+    if where == "host":
+        rng = np.random.default_rng(seed + 7919)
+        dout = _host_normal(rng, (B, h, d))
+        u = rng.uniform(0.05, 1.0, (B, h, 1, ms))
+        u = u * (np.arange(ms)[None, None, None, :] < lens[:, None, None, None])
+        tot = u.sum(axis=3, keepdims=True)
+        w = np.divide(u, tot, out=np.zeros_like(u), where=tot > 0)
+        return dict(dout=dout, weights=f32_to_bf16_bits(w.astype(np.float32)))
+    import torch
+    dout = _device_normal((B, h, d), seed, 4)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(int(seed) * 1000003 + 5)
+    u = torch.rand((B, h, 1, ms), generator=g, device="cuda") * 0.95 + 0.05
+    ln = torch.as_tensor(lens, device="cuda")
+    u = u * (torch.arange(ms, device="cuda")[None, None, None, :] < ln[:, None, None, None])
+    tot = u.sum(dim=3, keepdim=True)
+    w = torch.where(tot > 0, u / tot.clamp_min(1e-30), torch.zeros_like(u))
+    return dict(dout=dout, weights=w.to(torch.bfloat16))
