@@ -43,7 +43,6 @@ EXPORTS = {
     "attn_smallseq_fwd": (_I, [_P] * 4 + [_I] * 5 + [_F, _P, _P, _P]),
     "attn_smallseq_bwd": (_I, [_P] * 6 + [_I] * 5 + [_F, _P, _P, _P, _P]),
     "attn_get_last_device_error": (_I, [_P]),
-    "attn_selftest_exp2": (_I, [_P, _P, _I, _P]),
 }
 for _name, (_res, _args) in EXPORTS.items():
     _fn = getattr(lib, _name)
@@ -108,14 +107,6 @@ def attn_get_last_device_error(stream=None):
     if rc < 0:
         raise AttnError("attn_get_last_device_error", rc)
     return rc
-
-
-def attn_selftest_exp2(x, stream=None):
-    """The prefill's FMA-pipe 2^x approximation applied to a float32 CUDA tensor."""
-    _need(x, "x", torch.float32)
-    y = torch.empty_like(x)
-    _check("attn_selftest_exp2", lib.attn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
-    return y
 
 
 def attn_varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_q, max_k, causal=True, scale=None,

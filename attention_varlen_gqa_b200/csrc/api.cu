@@ -495,15 +495,6 @@ int attn_smallseq_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v
   return launch_smallseq_bwd(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
 }
 
-int attn_selftest_exp2(const float *x, float *y, int n, attn_stream_t stream) {
-  if (n < 0) return ATTN_E_SHAPE;
-  if (n > 0 && (!x || !y)) return ATTN_E_NULL;
-  unsigned int *err = nullptr;
-  int rc = device_state(&err);
-  if (rc) return rc;
-  return launch_exp2_selftest(x, y, n, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK
-                                                                                       : ATTN_E_CUDA;
-}
 
 int attn_get_last_device_error(attn_stream_t stream) {
   unsigned int *err = nullptr;

@@ -85,39 +85,6 @@ ATTN_DEVICE float max3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe for two values at once (x <= 2^20; inputs below -125
-// are treated as -125, so results are never below ~1.7e-38 and never zero).  Cody-Waite split x = n + f with n = round(x) taken
-// from the low mantissa bits of x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f from a
-// cubic whose coefficients minimise the maximum relative error on that
-// interval (7.5e-5; fitted by attention_varlen_gqa_b200/fit_exp2_poly.py);
-// 2^n is added to the exponent field.  Used for part of the softmax
-// exponentials so that the MUFU unit is not the only exp pipe.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
-constexpr float kExp2Round = 12582912.0f;   // 1.5 * 2^23
-
-ATTN_DEVICE uint64_t exp2_poly_x2(uint64_t x2) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -125.f);     // keeps n >= -125, so every result is a normal float
-  x1 = fmaxf(x1, -125.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t y = f2_add(x, f2_pack(kExp2Round, kExp2Round));        // round(x) in the low bits
-  const uint64_t n = f2_add(y, f2_pack(-kExp2Round, -kExp2Round));      // round(x) as a float
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);                  // x - round(x)
-  uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
-  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
-  float q0, q1, y0, y1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(y, y0, y1);
-  const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(y0) << 23));
-  const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(y1) << 23));
-  return f2_pack(r0, r1);
-}
-
 // ---------------------------------------------------------------------------
 // warp-level bf16 MMA (m16n8k16, fp32 accumulate) and ldmatrix
 // ---------------------------------------------------------------------------

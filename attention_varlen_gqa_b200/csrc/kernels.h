@@ -68,7 +68,6 @@ cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream);
 cudaError_t launch_smallseq_bwd(const SmallSeqParams &p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);
-cudaError_t launch_exp2_selftest(const float *x, float *y, int n, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap,
                            const CUtensorMap &kmap, const CUtensorMap &vmap, const CUtensorMap &omap,
                            cudaStream_t stream);

@@ -958,28 +958,7 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUte
   return cudaGetLastError();
 }
 
-__global__ void exp2_selftest_kernel(const float *x, float *y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    float a, b;
-    f2_unpack(exp2_poly_x2(f2_pack(x[i], x[i + 1])), a, b);
-    y[i] = a;
-    y[i + 1] = b;
-  } else if (i < n) {
-    float a, b;
-    f2_unpack(exp2_poly_x2(f2_pack(x[i], 0.f)), a, b);
-    y[i] = a;
-  }
-}
-
 }  // namespace
-
-cudaError_t launch_exp2_selftest(const float *x, float *y, int n, cudaStream_t stream) {
-  if (n <= 0) return cudaSuccess;
-  const int pairs = (n + 1) / 2;
-  exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
                            const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t stream) {

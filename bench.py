@@ -51,10 +51,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip", "smallseq_bwd"],
+                    default="all",
                     help="profiling aid: run a single operation (no JSON line)")
     ap.add_argument("--no-skip", action="store_true",
-                    help="leave out the skip-softmax and paged-prefill measurements")
+                    help="leave out the skip-softmax, paged-prefill and small-seq backward measurements")
     ap.add_argument("--no-cpu", action="store_true", help="leave out the CPU oracle baseline")
     ap.add_argument("--small", action="store_true",
                     help="profiling aid with --only: quarter-size decode / small-seq batches")
@@ -336,6 +337,11 @@ def main():
     if args.only == "skip":
         measure_skip(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
         return
+    if args.only == "smallseq_bwd":
+        measure_smallseq_bwd(A, W, torch, dev, seed, pk, reps=max(1, args.steps),
+                             batch=7680 if args.small else 30720)
+        assert A.attn_get_last_device_error() == 0
+        return
 
     def barrier():
         if world > 1:
@@ -409,10 +415,11 @@ def main():
     agg = aggregate_ranks({"per": per, "total_ms": total_ms, "e2e_ms": e2e_ms_local, "flops": pre_flops,
                            "dec_bytes": dec_bytes, "ss_bytes": ss_bytes}, world, dev)
 
-    skip = paged = None
+    skip = paged = ssb = None
     if not args.no_skip:
         skip = measure_skip(A, W, torch, dev, seed, pk, reps=3)
         paged = measure_paged_prefill(A, W, torch, dev, seed, pk, reps=3)
+        ssb = measure_smallseq_bwd(A, W, torch, dev, seed, pk, reps=5)
 
     if rank != 0:
         if world > 1:
@@ -460,6 +467,7 @@ def main():
         "rows": rows,
         "skip": skip,
         "paged_prefill": paged,
+        "smallseq_bwd": ssb,
         "cpu_baseline": cpu,
         "e2e": {"value": agg["e2e_value"], "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": agg["e2e_ms"],
@@ -569,6 +577,38 @@ def measure_paged_prefill(A, W, torch, dev, seed, pk, reps=3):
                         "h 32/8, d 128, page 16, causal",
             "ms": ms, "flops": flops, "tflops": flops / ms / 1e9, "frac_of_measured": flops / ms / 1e9 / pk["bf16"],
             "lens_k": [int(x) for x in lens_k]}
+
+
+def measure_smallseq_bwd(A, W, torch, dev, seed, pk, reps=5, batch=30720):
+    """Small-seq backward on the small-seq step workload (30720 tokens, s_kv
+    from {2,4,6,8,12,16}, h 16, d 128) with dO ~ N(0, 1) and synthetic saved
+    weights; inputs and outputs (4.4 GB) exceed L2.  Not a step row: reported
+    beside it.  Bytes: q, dO, K, V, weights read; dq, dK, dV written."""
+    s = W.smallseq(seed=seed, batch=batch, where="device")
+    g = W.smallseq_grad_inputs(s, seed=seed, where="device")
+    cu = torch.from_numpy(s["cu_seqlens_kv"]).to(dev)
+    q, k, v = s["q"], s["k"], s["v"]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def run():
+        A.attn_smallseq_bwd(q, k, v, g["dout"], g["weights"], cu, s["max_s_kv"], dq=dq, dk=dk, dv=dv)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    byts = (3 * q.numel() + 4 * k.numel() + g["weights"].numel()) * 2
+    gbs = byts / ms / 1e6
+    return {"workload": f"{batch} x s_kv{{2..16}} seed 0, h 16, d 128; dO, synthetic saved weights",
+            "ms": ms, "bytes": byts, "gbs": gbs, "frac_of_measured": gbs / pk["hbm"],
+            "frac_of_8000": gbs / 8000.0,
+            "traffic": recorded_traffic("smallseq_bwd_b30720", source_hash("smallseq.cu", "common.cuh"),
+                                        "bytes", byts)}
 
 
 if __name__ == "__main__":

@@ -355,15 +355,6 @@ ATTN_API int attn_smallseq_bwd(const attn_bf16 *q, const attn_bf16 *k, const att
                                attn_bf16 *dv, attn_stream_t stream);
 
 /*
- * attn_selftest_exp2 -- diagnostic: y[i] = the FMA-pipe approximation of 2^x[i]
- * that the prefill softmax uses for part of its exponentials (Cody-Waite split
- * plus a cubic on [-1/2, 1/2], maximum relative error 7.5e-5 for x in
- * [-125, 2^20]; inputs below -125 are treated as -125).  x and y are n device
- * floats.  Exists so tests can compare it with the CUDA math library.
- */
-ATTN_API int attn_selftest_exp2(const float *x, float *y, int n, attn_stream_t stream);
-
-/*
  * attn_get_last_device_error -- synchronises `stream`, then returns and
  * clears the current device's error word (a mask of ATTN_DEVERR_* bits), or
  * a negative ATTN_E_CUDA if the synchronisation itself failed.
