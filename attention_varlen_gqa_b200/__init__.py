@@ -40,6 +40,7 @@ EXPORTS = {
     "attn_paged_decode": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _S, _P]),
     "attn_paged_decode_ex": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _P, _P, _S, _P]),
     "attn_paged_decode_static": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P]),
+    "attn_paged_decode_workspace_size_ex": (_S, [_I, _I, _I, _I, _F]),
     "attn_smallseq_fwd": (_I, [_P] * 4 + [_I] * 5 + [_F, _P, _P, _P]),
     "attn_smallseq_bwd": (_I, [_P] * 6 + [_I] * 5 + [_F, _P, _P, _P, _P]),
     "attn_get_last_device_error": (_I, [_P]),
@@ -176,15 +177,20 @@ def prefill_skip_mask_words(batch, max_q, max_k, h_q, block_m=128, skip_tile=32)
     return -(-(batch * qb * h_q * kt) // 32), qb, kt
 
 
-def attn_paged_decode_workspace_size(batch, h_q, d):
+def attn_paged_decode_workspace_size(batch, h_q, d, max_pages_per_seq=0, skip_threshold=0.0):
+    if skip_threshold > 0.0:
+        return int(lib.attn_paged_decode_workspace_size_ex(batch, h_q, d, max_pages_per_seq, float(skip_threshold)))
     return int(lib.attn_paged_decode_workspace_size(batch, h_q, d))
 
 
 def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size=16, skip_threshold=0.0,
                       scale=None, out=None, lse=None, workspace=None, skip_mask=None,
-                      skip_counts=None, want_lse=True, stream=None):
+                      skip_counts=None, want_lse=True, skip_schedule="split", stream=None):
     """One-token paged decode. q [B, h_q, d]; caches [pages, page_size, h_kv, d];
-    block_table int32 [B, max_pages]; seq_lens int32 [B].  Returns (out, lse)."""
+    block_table int32 [B, max_pages]; seq_lens int32 [B].  Returns (out, lse).
+    skip_schedule (skip_threshold > 0): "split" -- two passes over the split
+    schedule with a workspace (allocated here when not given); "sequential" --
+    one split per (sequence, kv-head), no workspace."""
     _need(q, "q", torch.bfloat16, 3)
     _need(k_cache, "k_cache", torch.bfloat16, 4)
     _need(v_cache, "v_cache", torch.bfloat16, 4)
@@ -199,8 +205,12 @@ def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size=16, 
     if lse is None and want_lse:
         lse = torch.empty((batch, h_q), dtype=torch.float32, device=q.device)
     ws_bytes = 0
-    if skip_threshold == 0.0:
-        need = attn_paged_decode_workspace_size(batch, h_q, d)
+    if skip_threshold > 0.0 and skip_schedule == "sequential":
+        workspace = None
+    elif skip_schedule not in ("split", "sequential"):
+        raise ValueError(f"skip_schedule must be 'split' or 'sequential', got {skip_schedule!r}")
+    else:
+        need = attn_paged_decode_workspace_size(batch, h_q, d, block_table.shape[1], skip_threshold)
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         ws_bytes = workspace.numel() * workspace.element_size()

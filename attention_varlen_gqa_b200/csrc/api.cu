@@ -283,6 +283,44 @@ size_t attn_paged_decode_workspace_size(int batch, int h_q, int d) {
   return align_up(rows * d * sizeof(float), 256) + align_up(rows * 2 * sizeof(float), 256);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Two-pass skip-mode workspace: the split partials, then the scores
+// [B, h_kv, s_stride, G], the 32-key tile maxima [B, h_kv, kt_max, G] and the
+// split maxima [B, h_kv, splits, G] (all fp32).
+struct SkipWorkspace {
+  size_t o, ml, s, tmax, smax, total;
+  int s_stride, kt_max;
+};
+
+SkipWorkspace skip_workspace(int batch, int h_q, int d, int max_pages_per_seq) {
+  SkipWorkspace w{};
+  const size_t rows = (size_t)batch * h_q * kDecodeSplits;
+  const long long keys = (long long)max_pages_per_seq * kPageSize;
+  w.s_stride = (int)((keys + 63) / 64 * 64);   // whole 64-key chunks
+  w.kt_max = (int)((keys + kSkipTile - 1) / kSkipTile);
+  w.o = 0;
+  w.ml = w.o + align_up(rows * d * sizeof(float), 256);
+  w.s = w.ml + align_up(rows * 2 * sizeof(float), 256);
+  w.tmax = w.s + align_up((size_t)batch * h_q * w.s_stride * sizeof(float), 256);
+  w.smax = w.tmax + align_up((size_t)batch * h_q * w.kt_max * sizeof(float), 256);
+  w.total = w.smax + align_up(rows * sizeof(float), 256);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_paged_decode_workspace_size_ex(int batch, int h_q, int d, int max_pages_per_seq,
+                                           float skip_threshold) {
+  if (!(skip_threshold > 0.f)) return attn_paged_decode_workspace_size(batch, h_q, d);
+  if (batch <= 0 || h_q <= 0 || d <= 0 || max_pages_per_seq <= 0) return 256;
+  return skip_workspace(batch, h_q, d, max_pages_per_seq).total;
+}
+
 int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
                          const int32_t *block_table, const int32_t *seq_lens,
                          int batch, int num_pages, int max_pages_per_seq, int page_size,
@@ -302,11 +340,15 @@ int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const att
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return ATTN_E_ALIGN;
   if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_E_TOO_LARGE;
-  const bool sequential = skip_threshold > 0.f;
-  if (!sequential && batch > 0) {
+  const bool skip = skip_threshold > 0.f;
+  // skip mode: two passes over the split schedule with a workspace, one
+  // sequential split per (sequence, kv-head) without
+  const bool two_pass = skip && workspace != nullptr;
+  if ((!skip || two_pass) && batch > 0) {
     if (!workspace) return ATTN_E_WORKSPACE;
     if (!aligned16(workspace)) return ATTN_E_ALIGN;
-    if (workspace_bytes < attn_paged_decode_workspace_size(batch, h_q, d)) return ATTN_E_WORKSPACE;
+    if (workspace_bytes < attn_paged_decode_workspace_size_ex(batch, h_q, d, max_pages_per_seq, skip_threshold))
+      return ATTN_E_WORKSPACE;
   }
   unsigned int *err = nullptr;
   rc = device_state(&err);
@@ -336,7 +378,17 @@ int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const att
   p.kt_max = (max_pages_per_seq * page_size + kSkipTile - 1) / kSkipTile;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.thr_log2 = thr_to_log2(skip_threshold);
-  p.sequential = sequential ? 1 : 0;
+  p.sequential = skip ? (two_pass ? 2 : 1) : 0;
+  if (two_pass && batch > 0) {
+    const SkipWorkspace w = skip_workspace(batch, h_q, d, max_pages_per_seq);
+    char *base = static_cast<char *>(workspace);
+    p.ws_o = reinterpret_cast<float *>(base + w.o);
+    p.ws_ml = reinterpret_cast<float *>(base + w.ml);
+    p.ws_s = reinterpret_cast<float *>(base + w.s);
+    p.ws_tmax = reinterpret_cast<float *>(base + w.tmax);
+    p.ws_smax = reinterpret_cast<float *>(base + w.smax);
+    p.s_stride = w.s_stride;
+  }
   p.err = err;
 
   if (skip_mask) {
@@ -410,8 +462,9 @@ int attn_paged_decode_static(const attn_bf16 *q, const attn_bf16 *k_cache, const
                              int num_pages, int max_pages_per_seq, int page_size, int h_q, int h_kv,
                              int d, float skip_threshold, float scale, attn_bf16 *out, float *lse,
                              attn_stream_t stream) {
-  if (batch < 0 || h_q < 1 || d < 1) return ATTN_E_SHAPE;
-  if (attn_paged_decode_workspace_size(batch, h_q, d) > ATTN_STATIC_WORKSPACE_BYTES)
+  if (batch < 0 || h_q < 1 || d < 1 || max_pages_per_seq < 0) return ATTN_E_SHAPE;
+  const bool skip = skip_threshold > 0.f;
+  if (!skip && attn_paged_decode_workspace_size(batch, h_q, d) > ATTN_STATIC_WORKSPACE_BYTES)
     return ATTN_E_TOO_LARGE;
   unsigned int *err = nullptr;
   int rc = device_state(&err);
@@ -419,9 +472,14 @@ int attn_paged_decode_static(const attn_bf16 *q, const attn_bf16 *k_cache, const
   void *scratch = nullptr;
   rc = static_scratch(&scratch);
   if (rc) return rc;
+  // skip mode: the two-pass schedule when its workspace fits the scratch array,
+  // else the sequential one, which needs none
+  if (skip && attn_paged_decode_workspace_size_ex(batch, h_q, d, max_pages_per_seq, skip_threshold) >
+                  ATTN_STATIC_WORKSPACE_BYTES)
+    scratch = nullptr;
   return attn_paged_decode_ex(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages,
                               max_pages_per_seq, page_size, h_q, h_kv, d, skip_threshold, scale,
-                              nullptr, nullptr, out, lse, scratch, ATTN_STATIC_WORKSPACE_BYTES,
+                              nullptr, nullptr, out, lse, scratch, scratch ? ATTN_STATIC_WORKSPACE_BYTES : 0,
                               stream);
 }
 

@@ -21,7 +21,7 @@
 // online-softmax state (m, l, O) over its tokens; the four are merged at the
 // end of the CTA.
 //
-// Dense schedule: K and V of a chunk travel together through a 3-stage ring
+// Dense schedule: K and V of a chunk travel together through a 2-stage ring
 // and every chunk is finished (S, softmax, PV) in the iteration it arrives.
 // Sequential skip schedule: two passes two chunks apart over a ring of chunk
 // slots, where a slot first receives a chunk's K and, once the score pass is
@@ -45,7 +45,10 @@ namespace {
 constexpr int kChunk = 64;              // tokens per chunk (4 pages)
 constexpr int kWarps = 4;               // 16 tokens of each chunk per warp
 constexpr int kThreads = 32 * kWarps;
-constexpr int kDenseStages = 3;         // dense: K+V chunks in the ring
+// dense: K+V chunks in the ring.  Two stages (66 KB) let three CTAs share an
+// SM: more warps to cover the per-chunk latencies than two CTAs with three
+// stages each, for the same bytes in flight (measured 0.736 vs 0.820 ms).
+constexpr int kDenseStages = 2;
 constexpr int kSeqSlots = 5;            // sequential: chunk slots; a slot holds a chunk's K, then its V
 constexpr int kSeqLookahead = 2;        // sequential: PV pass lags the score pass
 constexpr int kSeqRing = kSeqLookahead + 1;
@@ -559,6 +562,343 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                      ln);
 }
 
+// ===================== skip mode in two passes over the split schedule =====================
+// For thresholds <= 1 a skipped tile never raises the running max (every row
+// of it lies below the max), so the running max before a tile is the prefix
+// max of all earlier tiles' maxima whether they were kept or not.  The
+// decisions therefore follow from the tile maxima alone, and the sequential
+// walk can be replaced by two passes over the 32-split schedule:
+//   pass 1 (decode_scores_kernel): K of the split -> the group's scores
+//       (fp32, log2 domain) and the per-head maxima of every 32-key tile and
+//       of the whole split, written to the workspace;
+//   pass 2 (decode_skip_pv_kernel): the running max entering the split is the
+//       max of the earlier splits' maxima; walking its tiles in order, the
+//       split takes the same decisions as the sequential walk, copies the V
+//       pages and scores of kept tiles only, and leaves an (m, l, O) partial
+//       for decode_combine_kernel.
+// K is read once, V of kept tiles once, and the scores (4 bytes per key and
+// query head) are written and read once.
+
+// chunks in flight per CTA: two keep a pass-1 CTA at 36 KB and a pass-2 CTA at
+// 46 KB of shared memory, so five or four share an SM; the per-chunk work of
+// one CTA is latency-bound (barrier and dependency stalls), and more resident
+// warps hid it better than deeper rings (pass 2 at 5 stages: 0.69 ms under
+// ncu at 2 CTAs per SM; at 2 stages both passes 0.77 ms together)
+constexpr int kScoreStages = 2;      // pass 1: K chunks
+constexpr int kPvStages = 2;         // pass 2: V chunks (+ their scores)
+constexpr int kTmaxCap = 1024;       // pass 2: tile maxima of a split kept in shared memory
+
+template <int D, bool PV>
+struct PassLayout {
+  static constexpr int kStages = PV ? kPvStages : kScoreStages;
+  static constexpr int kSlot = kChunk * D * 2;                 // K (pass 1) or V (pass 2) of a chunk
+  static constexpr int kStage = kSlot + (PV ? kChunk * kMaxGroup * 4 : 0);   // + the chunk's scores
+  // pass 1: [2][warp][16] 16-key maxima; pass 2: [split][G] the earlier splits' maxima
+  static constexpr int kX = kStages * kStage;
+  static constexpr int kTmax = kX + kDecodeSplits * kMaxGroup * 4;   // pass 2: the split's tile maxima
+  static constexpr int kKeep = kTmax + (PV ? kTmaxCap * 4 : 0);  // pass 2: [stage] decision bits
+  static constexpr int kBar = kKeep + 8 * kStages;
+  static constexpr int kBt = kBar + kStages * 8;
+  static constexpr int kBtCap = 256;
+  static constexpr int kEnd = kBt + kBtCap * 4;
+  static constexpr int kMerge = kWarps * 16 * 4 * 2 + kWarps * 16 * D * 4;
+  static_assert(!PV || kMerge <= kStages * kStage, "merge area fits (pass 2 merges in the ring)");
+  static_assert(kStage % 1024 == 0, "stages keep the 128-byte swizzle alignment");
+  static constexpr size_t kBytes = 1024 + kEnd;
+};
+
+// The split's chunk range, the sequence length (0 when out of range) and its
+// block-table entries, validated and copied to shared memory when they fit.
+struct SplitRange {
+  int L, c0, c1;
+  const int32_t *pages;   // indexed by the sequence's page number
+  bool dead;              // a block-table entry of the range is out of bounds
+};
+
+// `extra(L, c0, c1)` runs before the block-table loads and before the barrier
+// that publishes them, so loads it issues share their round trip.
+template <typename Extra>
+ATTN_DEVICE SplitRange split_range(const DecodeParams &p, int b, int split, int32_t *bt_s, int bt_cap,
+                                   Extra extra) {
+  SplitRange r;
+  int L = __ldg(p.seq_lens + b);
+  const bool bad_len = (L < 0) | (L > p.max_pages * kPageSize);
+  if (bad_len) L = 0;
+  const int n_chunks_all = (L + kChunk - 1) / kChunk;
+  const int n128 = (L + kDecodeSplitTile - 1) / kDecodeSplitTile;
+  const int per = (n128 + kDecodeSplits - 1) / kDecodeSplits;
+  const int sub = kDecodeSplitTile / kChunk;
+  r.L = L;
+  r.c0 = min(n_chunks_all, split * per * sub);
+  r.c1 = min(n_chunks_all, (split + 1) * per * sub);
+  extra(L, r.c0, r.c1);
+  const int32_t *bt = p.block_table + (size_t)b * p.max_pages;
+  const int pg0 = r.c0 * (kChunk / kPageSize);
+  const int pg1 = r.c1 > r.c0 ? (min(L, r.c1 * kChunk) + kPageSize - 1) / kPageSize : pg0;
+  const bool local = pg1 - pg0 <= bt_cap;
+  bool bad_page = false;
+  for (int i = pg0 + (int)threadIdx.x; i < pg1; i += kThreads) {
+    const int pg = __ldg(bt + i);
+    bad_page |= (pg < 0) | (pg >= p.num_pages);
+    if (local) bt_s[i - pg0] = pg;
+  }
+  r.pages = local ? bt_s - pg0 : bt;
+  r.dead = __syncthreads_or(bad_page) != 0;
+  if (threadIdx.x == 0 && (r.dead || bad_len))
+    raise_error(p.err, r.dead ? ATTN_DEVERR_BLOCK_TABLE : ATTN_DEVERR_SEQ_LEN);
+  return r;
+}
+
+template <int D, int NH>
+__global__ void __launch_bounds__(kThreads) decode_scores_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                 DecodeParams p) {
+  using Lay = PassLayout<D, false>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(base);
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + Lay::kBar);
+  float *qx = reinterpret_cast<float *>(base + Lay::kX);
+  const int tid = threadIdx.x;
+  const Lane ln(tid);
+  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int G = p.group;
+  const SplitRange r = split_range(p, b, split, reinterpret_cast<int32_t *>(base + Lay::kBt), Lay::kBtCap,
+                                   [](int, int, int) {});
+  const int n = r.c1 - r.c0;
+  const size_t seq = (size_t)b * p.h_kv + hk;
+  float *S = p.ws_s + seq * (size_t)p.s_stride * G;          // [token][G]
+  float *tmax = p.ws_tmax + seq * (size_t)p.kt_max * G;     // [tile][G]
+  float smax = -INFINITY;   // thread (tt, h) = tid (tt * G + h): head h's max over tiles tt of each chunk
+  if (!r.dead && n > 0) {
+    if (tid == 0) {
+      tma_prefetch_desc(&kmap);
+      for (int s = 0; s < Lay::kStages; ++s) mbar_init(&full[s], 1);
+      fence_barrier_init();
+    }
+    uint32_t qb[NH][D / 16][2];
+    load_q_frags<D, NH>(qb, p.q + ((size_t)b * p.h_q + (size_t)hk * G) * D, G, ln);
+    __syncthreads();
+    int issued = 0;
+    auto issue = [&](int c) {
+      const int s = c % Lay::kStages;
+      issue_pages<D>(&kmap, base + s * Lay::kStage, &full[s], r.pages, (r.c0 + c) * kChunk, r.L, hk, 0, 4,
+                     true);
+    };
+    if (tid == 0)
+      for (; issued < min(n, Lay::kStages); ++issued) issue(issued);
+    bool failed = false;
+    for (int i = 0; i < n; ++i) {
+      const int s = i % Lay::kStages;
+      const bool ok = mbar_wait(&full[s], (i / Lay::kStages) & 1, p.err);
+      if (ok) {
+        const int tok_base = (r.c0 + i) * kChunk + ln.w * 16;
+        float sc[NH][4], qm[NH][2];
+        warp_scores<D, NH>(sc, qm, sbase + s * Lay::kStage, qb, tok_base, r.L, G, p.scale_log2, ln);
+#pragma unroll
+        for (int nn = 0; nn < NH; ++nn) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = tok_base + ln.g + 8 * (e >> 1);
+            const int h = 8 * nn + ln.cq + (e & 1);
+            if (t < r.L && h < G) S[(size_t)t * G + h] = sc[nn][e];
+          }
+          if (ln.g == 0) {
+            qx[((i & 1) * kWarps + ln.w) * 16 + 8 * nn + ln.cq] = qm[nn][0];
+            qx[((i & 1) * kWarps + ln.w) * 16 + 8 * nn + ln.cq + 1] = qm[nn][1];
+          }
+        }
+      }
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      // every warp is done with stage s; chunk i's 16-key maxima are visible
+      if (tid == 0 && issued < n) issue(issued++);
+      if (tid < 2 * G) {
+        const int tt = tid / G, h = tid % G;
+        const float *x = qx + (i & 1) * kWarps * 16;
+        const float tm = fmaxf(x[(2 * tt) * 16 + h], x[(2 * tt + 1) * 16 + h]);
+        const int tile = 2 * (r.c0 + i) + tt;
+        if (tile * kSkipTile < r.L) tmax[(size_t)tile * G + h] = tm;
+        smax = fmaxf(smax, tm);
+      }
+    }
+    if (failed && tid == 0)
+      for (int x = issued - min(Lay::kStages, issued); x < issued; ++x)
+        mbar_wait(&full[x % Lay::kStages], (x / Lay::kStages) & 1, nullptr);
+  }
+  if (tid < 32) {
+    // lanes h and G + h hold head h's maxima over the chunks' first and second tiles
+    const float other = __shfl_sync(0xffffffffu, smax, (tid + G) & 31);
+    if (tid < G) p.ws_smax[(seq * kDecodeSplits + split) * G + tid] = fmaxf(smax, other);
+  }
+}
+
+template <int D, int NH>
+__global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_constant__ CUtensorMap vmap,
+                                                                  DecodeParams p) {
+  using Lay = PassLayout<D, true>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(base);
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + Lay::kBar);
+  float *tm_s = reinterpret_cast<float *>(base + Lay::kTmax);
+  uint32_t *keep_s = reinterpret_cast<uint32_t *>(base + Lay::kKeep);
+  const int tid = threadIdx.x;
+  const Lane ln(tid);
+  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int G = p.group;
+  const size_t seq = (size_t)b * p.h_kv + hk;
+  const float *S = p.ws_s + seq * (size_t)p.s_stride * G;
+  const float *tmax = p.ws_tmax + seq * (size_t)p.kt_max * G;
+
+  // with the block-table entries, in the same round trip: the split's tile
+  // maxima and the earlier splits' maxima, to shared memory
+  float *sm_s = reinterpret_cast<float *>(base + Lay::kX);   // [split][G], earlier splits
+  const SplitRange r = split_range(
+      p, b, split, reinterpret_cast<int32_t *>(base + Lay::kBt), Lay::kBtCap, [&](int L, int c0, int c1) {
+        const int nt = max(0, min((L + kSkipTile - 1) / kSkipTile, 2 * c1) - 2 * c0);
+        const int ntm = (2 * (c1 - c0) * G <= kTmaxCap) ? nt * G : 0;
+        const int nsm = split * G;
+        const float *tsrc = tmax + (size_t)2 * c0 * G;
+        const float *ssrc = p.ws_smax + seq * kDecodeSplits * G;
+        const float a = tid < ntm ? tsrc[tid] : 0.f;
+        const float c = tid < nsm ? ssrc[tid] : 0.f;
+        if (tid < ntm) tm_s[tid] = a;
+        if (tid < nsm) sm_s[tid] = c;
+        for (int x = tid + kThreads; x < ntm; x += kThreads) tm_s[x] = tsrc[x];
+        for (int x = tid + kThreads; x < nsm; x += kThreads) sm_s[x] = ssrc[x];
+      });
+  const int n = r.c1 - r.c0;
+  const bool tm_local = 2 * n * G <= kTmaxCap;
+
+  float o_acc[D / 16][NH][4];
+  float m_w[NH][2], l_w[NH][2];
+#pragma unroll
+  for (int nn = 0; nn < NH; ++nn) {
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o_acc[t][nn][e] = 0.f;
+    m_w[nn][0] = m_w[nn][1] = -INFINITY;
+    l_w[nn][0] = l_w[nn][1] = 0.f;
+  }
+  bool failed = false;
+  if (!r.dead && n > 0) {
+    if (tid == 0) {
+      tma_prefetch_desc(&vmap);
+      for (int s = 0; s < Lay::kStages; ++s) mbar_init(&full[s], 1);
+      fence_barrier_init();
+    }
+    // warp 0 takes the decisions (lane h: head h) and issues the copies
+    const bool head = ln.lane < G;
+    float m_run = -INFINITY;   // head lane's running max entering the next tile
+    unsigned long long n_vis = 0, n_skip = 0;
+    if (ln.w == 0 && head)
+      for (int s2 = 0; s2 < split; ++s2) m_run = fmaxf(m_run, sm_s[s2 * G + ln.lane]);
+    __syncthreads();   // barrier init
+    auto decide = [&](int c) -> uint32_t {
+      uint32_t kb = 0;
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        const int tile = 2 * (r.c0 + c) + tt;
+        const bool vis = tile * kSkipTile < r.L;
+        const float tm = (vis && head) ? (tm_local ? tm_s[(2 * c + tt) * G + ln.lane]
+                                                   : tmax[(size_t)tile * G + ln.lane])
+                                       : -INFINITY;
+        // a head votes skip when exp(tile max - running max) < threshold
+        const bool vote = !head || tm == -INFINITY || (tm - m_run < p.thr_log2);
+        m_run = fmaxf(m_run, tm);
+        const bool kept = vis && !__all_sync(0xffffffffu, vote);
+        if (kept) kb |= 1u << tt;
+        if (vis) {
+          ++n_vis;
+          if (!kept) {
+            ++n_skip;
+            if (p.skip_mask && ln.lane == 0) {
+              const long long unit = (long long)seq * p.kt_max + tile;
+              atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
+            }
+          }
+        }
+      }
+      return kb;
+    };
+    auto issue = [&](int c, uint32_t kb) {   // lane 0 of warp 0
+      const int s = c % Lay::kStages;
+      uint8_t *stage = base + s * Lay::kStage;
+      const int tok0 = (r.c0 + c) * kChunk;
+      const int npg = (min(r.L - tok0, kChunk) + kPageSize - 1) / kPageSize;
+      // pages 0-1 hold tile A, 2-3 tile B
+      const int lo = (kb & 1u) ? 0 : ((kb & 2u) ? 2 : 4);
+      const int hi = min(npg, (kb & 2u) ? 4 : ((kb & 1u) ? 2 : 0));
+      const uint32_t sbytes = kb ? kChunk * G * 4 : 0u;
+      keep_s[s] = kb;
+      mbar_arrive_expect_tx(&full[s], max(0, hi - lo) * (D / 64) * (16 * 64 * 2) + sbytes);
+      issue_pages<D>(&vmap, stage, &full[s], r.pages, tok0, r.L, hk, lo, hi, false);
+      if (sbytes) bulk_load(stage + Lay::kSlot, S + (size_t)tok0 * G, sbytes, &full[s]);
+    };
+    int issued = 0;
+    if (ln.w == 0)
+      for (; issued < min(n, Lay::kStages); ++issued) {
+        const uint32_t kb = decide(issued);
+        if (ln.lane == 0) issue(issued, kb);
+      }
+    for (int i = 0; i < n; ++i) {
+      const int s = i % Lay::kStages;
+      const bool ok = mbar_wait(&full[s], (i / Lay::kStages) & 1, p.err);
+      if (ok) {
+        const uint32_t kb = keep_s[s];
+        const int tok_base = (r.c0 + i) * kChunk + ln.w * 16;
+        if (((kb >> (ln.w >> 1)) & 1u) && tok_base < r.L) {
+          const uint32_t vslot = sbase + s * Lay::kStage;
+          const float *ss = reinterpret_cast<const float *>(base + s * Lay::kStage + Lay::kSlot);
+          float sc[NH][4], qm[NH][2];
+#pragma unroll
+          for (int nn = 0; nn < NH; ++nn) {
+            qm[nn][0] = qm[nn][1] = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int tl = ln.w * 16 + ln.g + 8 * (e >> 1);
+              const int h = 8 * nn + ln.cq + (e & 1);
+              const float v = (tok_base - ln.w * 16 + tl < r.L && h < G) ? ss[tl * G + h] : -INFINITY;
+              sc[nn][e] = v;
+              qm[nn][e & 1] = fmaxf(qm[nn][e & 1], v);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int o = 4; o < 32; o <<= 1)
+                qm[nn][h] = fmaxf(qm[nn][h], __shfl_xor_sync(0xffffffffu, qm[nn][h], o));
+          }
+          zero_tail_rows<D>(base, vslot, tok_base, r.L, ln);
+          warp_pv<D, NH>(o_acc, m_w, l_w, sc, qm, vslot, ln);
+        }
+      }
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      // every warp is done with stage s
+      if (ln.w == 0 && issued < n) {
+        const uint32_t kb = decide(issued);
+        if (ln.lane == 0) issue(issued, kb);
+        ++issued;
+      }
+    }
+    if (failed && tid == 0)
+      for (int x = issued - min(Lay::kStages, issued); x < issued; ++x)
+        mbar_wait(&full[x % Lay::kStages], (x / Lay::kStages) & 1, nullptr);
+    if (tid == 0 && p.skip_counts) {
+      atomicAdd(p.skip_counts + 0, n_vis);
+      atomicAdd(p.skip_counts + 1, n_skip);
+    }
+    __syncthreads();
+  }
+  merge_and_store<D, NH>(base, o_acc, m_w, l_w, r.dead || failed, G, b, hk, split, kDecodeSplits, false, p,
+                         ln);
+}
+
 // One warp per (sequence, q-head): log-sum-exp combine of the 32 split partials.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
@@ -610,11 +950,29 @@ cudaError_t launch_g(const DecodeParams &p, const CUtensorMap &kmap, const CUten
   return p.group <= 8 ? launch_k<D, SEQ, 1>(p, kmap, vmap, stream) : launch_k<D, SEQ, 2>(p, kmap, vmap, stream);
 }
 
+template <int D, int NH>
+cudaError_t launch_two_pass(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                            cudaStream_t stream) {
+  const size_t s1 = PassLayout<D, false>::kBytes, s2 = PassLayout<D, true>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(decode_scores_kernel<D, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)s1);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(decode_skip_pv_kernel<D, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
+  if (e != cudaSuccess) return e;
+  dim3 grid(kDecodeSplits, p.h_kv, p.batch);
+  decode_scores_kernel<D, NH><<<grid, kThreads, s1, stream>>>(kmap, p);
+  decode_skip_pv_kernel<D, NH><<<grid, kThreads, s2, stream>>>(vmap, p);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_d(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
-  if (p.sequential) return launch_g<D, true>(p, kmap, vmap, stream);
-  cudaError_t e = launch_g<D, false>(p, kmap, vmap, stream);
+  if (p.sequential == 1) return launch_g<D, true>(p, kmap, vmap, stream);
+  cudaError_t e = p.sequential == 2
+                      ? (p.group <= 8 ? launch_two_pass<D, 1>(p, kmap, vmap, stream)
+                                      : launch_two_pass<D, 2>(p, kmap, vmap, stream))
+                      : launch_g<D, false>(p, kmap, vmap, stream);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)p.batch * p.h_q;
   decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);

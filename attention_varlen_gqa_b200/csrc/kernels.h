@@ -35,14 +35,18 @@ struct DecodeParams {
   const int32_t *seq_lens;      // [B]
   uint16_t *out;                // [B, h_q, d]
   float *lse;                   // [B, h_q] or null
-  float *ws_o;                  // [B, h_q, splits, d]   (dense schedule)
-  float *ws_ml;                 // [B, h_q, splits, 2]   (dense schedule)
+  float *ws_o;                  // [B, h_q, splits, d]   (split schedules)
+  float *ws_ml;                 // [B, h_q, splits, 2]   (split schedules)
+  float *ws_s;                  // [B, h_kv, max_pages * 16, G] scores (two-pass skip)
+  float *ws_tmax;               // [B, h_kv, kt_max, G] 32-key tile maxima (two-pass skip)
+  float *ws_smax;               // [B, h_kv, splits, G] split maxima (two-pass skip)
   uint32_t *skip_mask;          // or null
   unsigned long long *skip_counts;  // or null
   int batch, h_q, h_kv, group, d, num_pages, max_pages, kt_max;
+  int s_stride;                 // key slots per (sequence, kv-head) in ws_s: max_pages * 16 rounded up to 64
   float scale_log2;             // scale * log2(e)
   float thr_log2;               // log2(threshold); -inf when skipping is off
-  int sequential;               // 1: one split walking 32-key tiles (skip mode)
+  int sequential;               // skip mode: 1 = one split walking 32-key tiles, 2 = two passes
   unsigned int *err;
 };
 

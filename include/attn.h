@@ -222,6 +222,17 @@ ATTN_API int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, co
 ATTN_API size_t attn_paged_decode_workspace_size(int batch, int h_q, int d);
 
 /*
+ * attn_paged_decode_workspace_size_ex -- the same query for either schedule:
+ * skip_threshold == 0 gives attn_paged_decode_workspace_size(batch, h_q, d);
+ * skip_threshold > 0 gives the two-pass skip schedule's need: the split
+ * partials plus, in float32, the scores of every (query head, key slot up to
+ * max_pages_per_seq * 16, rounded up to 64), the maxima of every 32-key tile
+ * and of every split (about batch * h_q * max_pages_per_seq * 64 bytes).
+ */
+ATTN_API size_t attn_paged_decode_workspace_size_ex(int batch, int h_q, int d, int max_pages_per_seq,
+                                                    float skip_threshold);
+
+/*
  * attn_paged_decode -- one query token per sequence against a paged cache.
  *
  *   q              [batch, h_q, d] bf16
@@ -235,14 +246,22 @@ ATTN_API size_t attn_paged_decode_workspace_size(int batch, int h_q, int d);
  *   page_size      16
  *   skip_threshold 0: dense split-KV schedule (32 splits of 128-key tiles per
  *                  (sequence, kv-head)) followed by a log-sum-exp combine;
- *                  > 0 (and <= 1): one sequential split per (sequence,
- *                  kv-head) walking 32-key tiles; a tile is skipped when all
- *                  h_q / h_kv query heads of the group vote skip.
+ *                  > 0 (and <= 1): skip-softmax over 32-key tiles visited in
+ *                  order; a tile is skipped when all h_q / h_kv query heads
+ *                  of the group vote skip against the running max.  With a
+ *                  workspace this runs as two passes over the split schedule
+ *                  (scores and tile maxima, then the kept tiles' P V): a
+ *                  skipped tile never raises the running max, so the max
+ *                  entering a tile is the max of all earlier tiles and every
+ *                  split takes the sequential walk's decisions.  With
+ *                  workspace NULL it runs as one sequential split per
+ *                  (sequence, kv-head).  Both give the same decisions.
  *   out            [batch, h_q, d] bf16
  *   lse            [batch, h_q] float32, may be NULL
- *   workspace      device buffer of >= attn_paged_decode_workspace_size(...)
- *                  bytes, 16-byte aligned (needed only when skip_threshold
- *                  is 0; may be NULL otherwise)
+ *   workspace      device buffer of >= attn_paged_decode_workspace_size_ex(
+ *                  batch, h_q, d, max_pages_per_seq, skip_threshold) bytes,
+ *                  16-byte aligned; required when skip_threshold is 0, NULL
+ *                  (sequential skip schedule) or such a buffer otherwise
  */
 ATTN_API int attn_paged_decode(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
                       const int32_t *block_table, const int32_t *seq_lens,
@@ -280,10 +299,12 @@ ATTN_API int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, 
  * the workspace and keeps the split-KV partials in a scratch array that the
  * library itself holds in device memory:
  *
- *   - scratch limit: ATTN_STATIC_WORKSPACE_BYTES (48 MiB).  A shape whose
- *     attn_paged_decode_workspace_size(batch, h_q, d) exceeds it returns
- *     ATTN_E_TOO_LARGE and launches nothing (about batch * h_q <= 2900 at
- *     d = 128, <= 5600 at d = 64).
+ *   - scratch limit: ATTN_STATIC_WORKSPACE_BYTES (48 MiB).  A dense-mode
+ *     shape whose attn_paged_decode_workspace_size(batch, h_q, d) exceeds it
+ *     returns ATTN_E_TOO_LARGE and launches nothing (about batch * h_q <=
+ *     2900 at d = 128, <= 5600 at d = 64).  In skip mode the two-pass
+ *     schedule runs when its workspace fits the array, the sequential one
+ *     (no workspace) otherwise.
  *   - every GPU that loads the library reserves those 48 MiB until the
  *     process exits.
  *   - the first call on a device looks up the array's device address

@@ -65,6 +65,15 @@ def test_workspace_query(A):
     for B, h, d in ((64, 32, 128), (1, 1, 64), (7, 3, 128)):
         rows = B * h * 32
         assert A.attn_paged_decode_workspace_size(B, h, d) == align(rows * d * 4) + align(rows * 8)
+        # skip mode, two passes: + scores (key slots rounded up to 64), tile maxima, split maxima
+        for maxp in (1, 5, 2048):
+            slots = (maxp * 16 + 63) // 64 * 64
+            tiles = (maxp * 16 + 31) // 32
+            want = align(rows * d * 4) + align(rows * 8) + align(B * h * slots * 4) + align(B * h * tiles * 4) \
+                + align(rows * 4)
+            assert A.lib.attn_paged_decode_workspace_size_ex(B, h, d, maxp, 0.1) == want
+            assert A.lib.attn_paged_decode_workspace_size_ex(B, h, d, maxp, 0.0) == \
+                A.attn_paged_decode_workspace_size(B, h, d)
 
 
 FAKE = 1 << 20          # a 16-byte aligned fake address, never dereferenced
@@ -144,6 +153,9 @@ def test_decode_argument_errors(A):
     assert decode(A, wsb=100) == -9
     assert decode(A, ws=FAKE + 4) == -2
     assert decode(A, pages=0) == -8
+    # skip mode: a workspace selects the two-pass schedule and must be large enough
+    assert decode(A, thr=0.1, wsb=100) == -9
+    assert decode(A, thr=0.1, ws=FAKE + 4) == -2
 
 
 def smallseq(A, **kw):

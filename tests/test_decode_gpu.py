@@ -1,5 +1,6 @@
 """GPU parity: paged one-token decode (dense split-KV + combine, and the
-sequential skip-softmax schedule) against the oracle."""
+skip-softmax schedules: two passes over the splits, or one sequential split)
+against the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -29,7 +30,10 @@ def _dev(data):
     return t
 
 
-def _run(A, data, thr, t=None):
+SCHEDULES = ["split", "sequential"]
+
+
+def _run(A, data, thr, t=None, schedule="split"):
     t = t or _dev(data)
     B = len(data["seq_lens"])
     kt = -(-data["block_table"].shape[1] * 16 // 32)
@@ -37,7 +41,7 @@ def _run(A, data, thr, t=None):
     mask = torch.zeros(max(words, 1), dtype=torch.int32, device="cuda")
     counts = torch.zeros(2, dtype=torch.int64, device="cuda")
     out, lse = A.attn_paged_decode(t["q"], t["k_cache"], t["v_cache"], t["block_table"], t["seq_lens"],
-                                   skip_threshold=thr, skip_mask=mask, skip_counts=counts)
+                                   skip_threshold=thr, skip_mask=mask, skip_counts=counts, skip_schedule=schedule)
     return out, lse, mask, counts, kt
 
 
@@ -51,10 +55,10 @@ def _gpu_decisions(mask, kt, h_kv):
     return get
 
 
-def _check(A, data, thr, t=None, batches=None, host=None):
+def _check(A, data, thr, t=None, batches=None, host=None, schedule="split"):
     """Run on the GPU and compare with the oracle (optionally on sampled batches,
     with ``host`` giving host copies of the sampled sub-problem)."""
-    out, lse, mask, counts, kt = _run(A, data, thr, t)
+    out, lse, mask, counts, kt = _run(A, data, thr, t, schedule)
     assert A.attn_get_last_device_error() == 0
     h_q, h_kv = data["h_q"], data["h_kv"]
     if host is None:
@@ -114,22 +118,42 @@ def _peaked(lens, h_q=8, h_kv=2, d=128, seed=0):
     return data
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("thr", [1e-3, 1e-2, 0.1, 0.5, 0.9, 1.0])
-def test_skip_sets(A, thr):
+def test_skip_sets(A, thr, schedule):
     data = _peaked([1, 31, 33, 200, 700, 2048, 3000])
-    vis, skipped = _check(A, data, thr)
+    vis, skipped = _check(A, data, thr, schedule=schedule)
     assert vis > 0
     if thr >= 0.1:
         assert skipped > 0
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("heads", [(8, 1), (24, 2), (16, 1)])
-def test_skip_sets_wide_groups(A, heads):
+def test_skip_sets_wide_groups(A, heads, schedule):
     """Groups of 8, 12 and 16 query heads: one full, one partial and two full
     8-head column tiles of the decode MMAs."""
     data = _peaked([1, 33, 700, 3000], h_q=heads[0], h_kv=heads[1], seed=heads[0])
-    vis, _ = _check(A, data, 0.1)
+    vis, _ = _check(A, data, 0.1, schedule=schedule)
     assert vis > 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_schedules_agree(A, d):
+    """The two skip schedules take identical decisions (same mask and counts)
+    and give the same output within bf16 rounding, on long ragged sequences
+    whose splits span many tiles."""
+    data = _peaked([5, 64, 1000, 4097, 9000, 20000], d=d, seed=d)
+    t = _dev(data)
+    for thr in (0.05, 0.5):
+        o1, l1, m1, c1, _ = _run(A, data, thr, t, "split")
+        o2, l2, m2, c2, _ = _run(A, data, thr, t, "sequential")
+        assert A.attn_get_last_device_error() == 0
+        assert torch.equal(m1, m2) and torch.equal(c1, c2)
+        if thr >= 0.5:
+            assert int(c1[1]) > 0
+        assert torch.allclose(o1.float(), o2.float(), atol=2e-2, rtol=0)
+        assert torch.allclose(l1, l2, atol=1e-3, rtol=0)
 
 
 def test_skip_threshold_zero_is_dense(A):
@@ -143,13 +167,14 @@ def test_skip_threshold_zero_is_dense(A):
     assert torch.allclose(o0.float(), o1.float(), atol=2e-2)
 
 
-def test_bad_block_table_entry(A):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_bad_block_table_entry(A, schedule):
     data = W.paged_decode([40, 50], h_q=4, h_kv=2, d=128, seed=3)
     bt = data["block_table"].copy()
     bt[1, 2] = data["num_pages"] + 5
     data["block_table"] = bt
     for thr in (0.0, 0.1):
-        out, lse, _, _, _ = _run(A, data, thr)
+        out, lse, _, _, _ = _run(A, data, thr, schedule=schedule)
         assert A.attn_get_last_device_error() & 4
         assert torch.all(out[1] == 0)
         assert torch.all(torch.isneginf(lse[1]))
@@ -203,10 +228,11 @@ def test_full_size_dense_sampled(A):
     _check(A, data, 0.0, t=_dev(data), batches=batches, host=_sampled_host(data, batches))
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("thr", [1e-3, 1e-2, 0.1])
-def test_full_size_skip_sampled(A, thr):
+def test_full_size_skip_sampled(A, thr, schedule):
     """Batch 32 at 32768 keys with sink and window peaks; 3 sampled sequences
     vs the oracle, skip sets included."""
     data = W.skip_decode(seed=0, where="device")
     batches = [0, 13, 31]
-    _check(A, data, thr, t=_dev(data), batches=batches, host=_sampled_host(data, batches))
+    _check(A, data, thr, t=_dev(data), batches=batches, host=_sampled_host(data, batches), schedule=schedule)
