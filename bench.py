@@ -519,13 +519,20 @@ def measure_skip(A, W, torch, dev, seed, pk, reps=3):
     sl = torch.from_numpy(sd["seq_lens"]).to(dev)
     dout = torch.empty_like(sd["q"])
     dlse = torch.empty(sd["q"].shape[:2], dtype=torch.float32, device=dev)
-    ws = torch.empty(A.attn_paged_decode_workspace_size(32, 32, 128), dtype=torch.uint8, device=dev)
     Ls = sd["seq_lens"].astype(np.int64)
     kbytes = float(Ls.sum() * 8 * 128 * 2)
-    for thr in (0.0, 1e-3, 1e-2, 0.1):
+    # skip mode: the two-pass schedule (workspace given); "0.1/sequential" is the
+    # one-split-per-(sequence, kv-head) schedule at the same threshold
+    for key, thr, sched in ((0.0, 0.0, "split"), (1e-3, 1e-3, "split"), (1e-2, 1e-2, "split"),
+                            (0.1, 0.1, "split"), ("0.1/sequential", 0.1, "sequential")):
+        ws = None
+        if sched == "split":
+            ws = torch.empty(A.attn_paged_decode_workspace_size(32, 32, 128, bt.shape[1], thr), dtype=torch.uint8,
+                             device=dev)
+
         def run():
             A.attn_paged_decode(sd["q"], sd["k_cache"], sd["v_cache"], bt, sl, skip_threshold=thr,
-                                out=dout, lse=dlse, workspace=ws, skip_counts=counts)
+                                out=dout, lse=dlse, workspace=ws, skip_counts=counts, skip_schedule=sched)
         run()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -538,8 +545,10 @@ def measure_skip(A, W, torch, dev, seed, pk, reps=3):
         vis, sk = (int(x) for x in counts.tolist())
         frac = sk / vis if vis and thr > 0 else 0.0
         alg = kbytes + kbytes * (1.0 - frac) + 32 * 32 * 128 * 2 * 2 + 32 * 32 * 4
-        res["decode"][str(thr)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
-                                   "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"]}
+        res["decode"][str(key)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
+                                   "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"],
+                                   "schedule": "dense split-KV" if thr == 0 else
+                                   ("two passes over 32 splits" if sched == "split" else "one sequential split")}
     return res
 
 
