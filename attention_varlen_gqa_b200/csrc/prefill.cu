@@ -321,9 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = misc;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
   // skip votes of the four warps of a softmax warpgroup, per query tile and
-  // tile parity: bit u = every row of the warp votes to skip 32-key sub-tile u
-  volatile uint32_t *votes = misc + 4;          // [kNQ][2][4]
-  volatile int *ring = reinterpret_cast<volatile int *>(misc + 20);   // [kSchedDepth] claimed items
+  // tile count mod 3: bit u = every row of the warp votes to skip 32-key
+  // sub-tile u.  Three slots: a warp may reach tile c + 1 while a slower warp
+  // of its group still reads the votes of tile c - 1, but no warp writes tile
+  // c + 2's before every warp has handed over P of tile c + 1, which comes
+  // after that read.
+  volatile uint32_t *votes = misc + 4;          // [kNQ][3][4]
+  volatile int *ring = reinterpret_cast<volatile int *>(misc + 28);   // [kSchedDepth] claimed items
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = num_items(p);
@@ -490,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t kv_c = 0, q_c = 0;
     uint32_t tile_c[kNQ] = {0, 0};   // tiles processed per query-tile slot (p_full / o_done phases)
     uint32_t item_c[kNQ] = {0, 0};   // items with work per slot (o_free phases)
-    unsigned long long n_vis = 0, n_skip = 0;
+    uint32_t vslot[kNQ] = {0, 0};    // tile_c mod 3: the slot of the tile's votes
     bool ok = true;
     auto wait_all = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, p.err));
@@ -550,12 +554,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // every row votes for it, and its P.V MMAs (two 16-key steps) are not
           // issued.  The softmax warps take the skipped keys' p out of their
           // row sums one tile later.
-          uint32_t skip_bits = 0, vis_bits = 0;
-          if constexpr (SKIP) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) vis_bits |= uint32_t(j * BN + 32 * u < g[t].k_end) << u;
-            skip_bits = and4_shared(votes + (t * 2 + (tile_c[t] & 1)) * 4) & vis_bits;
-          }
+          // (sub-tiles past the keys vote skip too: their p is 0 either way)
+          uint32_t skip_bits = 0;
+          if constexpr (SKIP) skip_bits = and4_shared(votes + (t * 3 + vslot[t]) * 4);
           if (!v_ready) {
             if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
             tc_fence_after();
@@ -601,6 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pv_started[t] = __shfl_sync(0xffffffffu, acc, leader_lane);
           commit(&o_done[t]);
           ++tile_c[t];
+          vslot[t] = vslot[t] == 2 ? 0 : vslot[t] + 1;
           if (j + 1 < g[t].n) {
             if (!k_next_ready) {
               const uint32_t cn = c + 1;
@@ -609,23 +611,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               k_next_ready = true;
             }
             issue_s(t, (c + 1) % kStages);
-          }
-          // skip bookkeeping, after the MMAs are issued
-          if constexpr (SKIP) {
-            if (leader) {
-              n_vis += __popc(vis_bits);
-              n_skip += __popc(skip_bits);
-              if (p.skip_mask && skip_bits) {
-                for (int u = 0; u < 4; ++u) {
-                  if ((skip_bits >> u) & 1u) {
-                    const long long unit =
-                        (((long long)it.b * p.qb_max + it.r[t]) * p.h_q + it.hq[t]) * p.kt_max +
-                        (j * BN / 32 + u);
-                    atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
-                  }
-                }
-              }
-            }
           }
         }
         if (ok) commit(&kv_empty[st]);
@@ -636,10 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < kNQ; ++t) item_c[t] += g[t].n > 0 ? 1 : 0;
       kv_c += nmax;
       ++q_c;
-    }
-    if (SKIP && leader && p.skip_counts) {
-      atomicAdd(p.skip_counts + 0, n_vis);
-      atomicAdd(p.skip_counts + 1, n_skip);
     }
     // every MMA must be complete before the TMEM is released
 #pragma unroll
@@ -690,6 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t tile_c = 0;
     bool alive = true;
+    // skip-softmax counts of this warpgroup's units (kept by its first warp)
+    unsigned long long n_vis = 0, n_skip = 0;
 
     for (uint32_t n = 0; alive; ++n) {
       const int idx = pop_warp(n);
@@ -720,17 +703,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keys' p leave the row sum (their P.V MMAs were never issued)
       float ps[4] = {0.f, 0.f, 0.f, 0.f}, ps_prev[4] = {0.f, 0.f, 0.f, 0.f};
       // drop the skipped keys of the tile with warpgroup count c, local index
-      // jp, whose sub-tile sums are q, now worth `scale` each
+      // jp, whose sub-tile sums are q, now worth `scale` each; the first warp
+      // also counts and records the skipped units
       auto drop_skipped = [&](uint32_t c, int jp, const float (&q)[4], float scale) {
         alive = alive && __all_sync(0xffffffffu, wait_or_abort(&votes_ready[2 * t + (c & 1)], (c >> 1) & 1,
                                                                abort_flag, p.err));
-        const uint32_t skip = and4_shared(votes + (t * 2 + (c & 1)) * 4);
+        uint32_t skip = and4_shared(votes + (t * 3 + c % 3) * 4);
         float d = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (((skip >> u) & 1u) && jp * BN + 32 * u < g.k_end) d += q[u];
+        for (int u = 0; u < 4; ++u) {
+          const bool vis = jp * BN + 32 * u < g.k_end;
+          if (((skip >> u) & 1u) && vis) d += q[u];
+          if (!vis) skip &= ~(1u << u);
+        }
         l -= d * scale;
+        if (quad == 0 && skip != 0) {
+          n_skip += __popc(skip);
+          if (lane == 0 && p.skip_mask) {
+            for (int u = 0; u < 4; ++u) {
+              if ((skip >> u) & 1u) {
+                const long long unit = (((long long)it.b * p.qb_max + it.r[t]) * p.h_q + hq) * p.kt_max +
+                                       (jp * BN / 32 + u);
+                atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
+              }
+            }
+          }
+        }
       };
+      if (SKIP && quad == 0 && g.n > 0) n_vis += (g.k_end + kSkipTile - 1) / kSkipTile;
       auto step = [&](int j) -> bool {
         const bool ok =
             __all_sync(0xffffffffu, alive && wait_or_abort(&s_full[t], tile_c & 1, abort_flag, p.err));
@@ -750,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mref = (m_used == -INFINITY) ? 0.f : m_used;
         float um[4];                                // raw maxima of the four 32-key sub-tiles
         max_sub4(sr, um);
+        uint32_t wv = 0;                            // the warp's skip votes (bit u: sub-tile u)
         if constexpr (SKIP) {
           // vote per 32-key sub-tile: exp(sub-tile max - running max) <
           // threshold; the MMA warp combines the four warps' votes
@@ -761,10 +762,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_true = fmaxf(m_true, t2);
             my_votes |= uint32_t(vote) << u;
           }
-          const uint32_t wv = __reduce_and_sync(0xffffffffu, my_votes);
-          // the MMA warp reads it after the P hand-off below (which orders it);
-          // the warpgroup's own readers wait on votes_ready, arrived after it
-          if (lane == 0) votes[(t * 2 + (tile_c & 1)) * 4 + quad] = wv;
+          // stored with the P hand-off below (which orders it for the MMA
+          // warp; the warpgroup's own readers wait on votes_ready), so the
+          // reduction overlaps the exponentials
+          wv = __reduce_and_sync(0xffffffffu, my_votes);
         } else {
           m_true = fmaxf(m_true, fmaxf(fmaxf(um[0], um[1]), fmaxf(um[2], um[3])) * sl2);
         }
@@ -800,6 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
+          if (SKIP) votes[(t * 3 + tile_c % 3) * 4 + quad] = wv;
           mbar_arrive(&p_half[t]);
           if (SKIP) mbar_arrive(&votes_ready[2 * t + (tile_c & 1)]);
         }
@@ -912,6 +914,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[(size_t)(sq.q0 + i) * p.h_q + hq] = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
     }
     if (quad == 0 && lane == 0) bulk_wait_all();   // output boxes written before the CTA ends
+    if (SKIP && quad == 0 && lane == 0 && p.skip_counts) {
+      atomicAdd(p.skip_counts + 0, n_vis);
+      atomicAdd(p.skip_counts + 1, n_skip);
+    }
   }
 
   tc_fence_before();
