@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pv_started[t] = __shfl_sync(0xffffffffu, acc, leader_lane);
           commit(&o_done[t]);
           ++tile_c[t];
-          vslot[t] = vslot[t] == 2 ? 0 : vslot[t] + 1;
+          if constexpr (SKIP) vslot[t] = vslot[t] == 2 ? 0 : vslot[t] + 1;
           if (j + 1 < g[t].n) {
             if (!k_next_ready) {
               const uint32_t cn = c + 1;
