@@ -51,7 +51,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip", "smallseq_bwd"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip", "smallseq_bwd",
+                                       "decode_skip"],
                     default="all",
                     help="profiling aid: run a single operation (no JSON line)")
     ap.add_argument("--no-skip", action="store_true",
@@ -282,6 +283,8 @@ def main():
 
     # ---------------- inputs (device-resident) ----------------
     want = {"prefill", "decode", "smallseq"} if args.only == "all" else {args.only}
+    if args.only == "decode_skip":
+        want = {"decode"}
     ops = []
     if "prefill" in want:
         pre = W.gqa_prefill(seed=seed, where="device")
@@ -327,6 +330,16 @@ def main():
             A.attn_smallseq_fwd(ss["q"], ss["k"], ss["v"], ss_cu, 16, out=ss_out, weights=ss_w)
         ops.append(("smallseq", do_smallseq))
 
+    if args.only == "decode_skip":
+        # the decode workload in skip mode (threshold 0.1), two passes over the splits
+        dsk_ws = torch.empty(A.attn_paged_decode_workspace_size(dec_batch, 32, 128, dec["block_table"].shape[1], 0.1),
+                             dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup + args.steps):
+            A.attn_paged_decode(dec["q"], dec["k_cache"], dec["v_cache"], dec_bt, dec_sl, skip_threshold=0.1,
+                                out=dec_out, lse=dec_lse, workspace=dsk_ws)
+        torch.cuda.synchronize()
+        assert A.attn_get_last_device_error() == 0
+        return
     if args.only in ("prefill", "decode", "smallseq"):
         fn = dict(ops)[args.only]
         for _ in range(args.warmup + args.steps):
