@@ -587,3 +587,50 @@ def smallseq_backward(q, k, v, dout, weights, cu_seqlens_kv, h, scale, batches=N
             dq[b, hh] = scale * (dS @ kf[k0:k1, hh]) if n else 0.0   # grad_Q
             dk[k0:k1, hh] = scale * dS[:, None] * qf[b, hh][None, :]  # grad_K
     return dq, dk, dv
+
+
+def varlen_backward(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, h_q, h_kv, causal, scale, batches=None):
+    """Gradients of ``varlen_attention`` (dense, no skipping) w.r.t. q, k and v.
+
+    NVIDIA/Model-Optimizer PR 1034 "Add Triton unified attention kernel with
+    HuggingFace integration", description: the kernel serves training through
+    autograd, which needs the backward of the same masked softmax(Q K^T) V.
+    With P the row softmax over the allowed keys (recomputed here in fp64) and
+    dO the output gradient, the chain rule gives, per sequence and q-head
+    (kv-head hk = the q-head's group):
+      dV_hk += P^T dO                   dP = dO V^T
+      dS = P * (dP - rowsum(P * dP))    (rowsum(P * dP) = <dO_i, O_i>)
+      dQ = scale * dS K                 dK_hk += scale * dS^T Q
+    Rows with no allowed key have P = 0 and contribute nothing.
+
+    q, dout: [total_q, h_q, d]; k, v: [total_k, h_kv, d] (bf16 bits or float
+    values).  Returns fp64 dq, dk, dv; with ``batches`` only those sequences
+    are evaluated and the rest are NaN.
+    """
+    qf, kf, vf, of = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    cu_q = np.asarray(cu_seqlens_q, dtype=np.int64)
+    cu_k = np.asarray(cu_seqlens_k, dtype=np.int64)
+    B = len(cu_q) - 1
+    dq = np.full(qf.shape, np.nan)
+    dk = np.full(kf.shape, np.nan)
+    dv = np.full(vf.shape, np.nan)
+    for b in (range(B) if batches is None else batches):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
+        s_q, s_k = q1 - q0, k1 - k0
+        dk[k0:k1] = 0.0
+        dv[k0:k1] = 0.0
+        dq[q0:q1] = 0.0
+        if s_q == 0 or s_k == 0:
+            continue
+        allowed = allowed_mask(s_q, s_k, causal)
+        for hq in range(h_q):
+            hk = kv_head_of(hq, h_q, h_kv)
+            Q, K, V, dO = qf[q0:q1, hq], kf[k0:k1, hk], vf[k0:k1, hk], of[q0:q1, hq]
+            _, _, P = softmax_over_kept(scale * (Q @ K.T), allowed, V)
+            dv[k0:k1, hk] += P.T @ dO
+            dP = dO @ V.T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dq[q0:q1, hq] = scale * (dS @ K)
+            dk[k0:k1, hk] += scale * (dS.T @ Q)
+    return dq, dk, dv

@@ -576,6 +576,104 @@ def pin_smallseq_backward_single_key():
     close(dk, np.zeros_like(dk))
     close(dv, oracle.bf16_bits_to_f64(bf(do)))
 
+
+# ---------------------------------------------------------------------------
+# varlen backward
+# ---------------------------------------------------------------------------
+
+def _varlen_case(seed, lens_q, lens_k, h_q, h_kv, d):
+    rng = np.random.default_rng(seed)
+    cq, ck = cu_from_lens(np.asarray(lens_q)), cu_from_lens(np.asarray(lens_k))
+    q = rng.standard_normal((int(cq[-1]), h_q, d))
+    k = rng.standard_normal((int(ck[-1]), h_kv, d))
+    v = rng.standard_normal((int(ck[-1]), h_kv, d))
+    do = rng.standard_normal((int(cq[-1]), h_q, d))
+    return cq, ck, q, k, v, do
+
+
+def pin_varlen_backward_autograd():
+    """= torch autograd in fp64 of sum dO . O through the masked softmax, GQA
+    heads sharing one K/V leaf, causal (bottom-right, s_q < s_k included) and
+    not."""
+    h_q, h_kv, d, scale = 4, 2, 8, 0.35
+    lens_q, lens_k = [3, 9, 1, 6], [5, 9, 4, 6]
+    cq, ck, q, k, v, do = _varlen_case(17, lens_q, lens_k, h_q, h_kv, d)
+    for causal in (True, False):
+        dq, dk, dv = oracle.varlen_backward(q, k, v, do, cq, ck, h_q, h_kv, causal, scale)
+        qt = torch.tensor(q, requires_grad=True)
+        kt = torch.tensor(k, requires_grad=True)
+        vt = torch.tensor(v, requires_grad=True)
+        loss = 0.0
+        for b in range(len(lens_q)):
+            q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+            s_q, s_k = q1 - q0, k1 - k0
+            i = torch.arange(s_q)[:, None]
+            j = torch.arange(s_k)[None, :]
+            mask = (j <= i + (s_k - s_q)) if causal else torch.ones(s_q, s_k, dtype=torch.bool)
+            for hq in range(h_q):
+                hk = hq // (h_q // h_kv)
+                S = scale * (qt[q0:q1, hq] @ kt[k0:k1, hk].T)
+                P = torch.softmax(S.masked_fill(~mask, float("-inf")), dim=1)
+                loss = loss + (torch.tensor(do[q0:q1, hq]) * (P @ vt[k0:k1, hk])).sum()
+        loss.backward()
+        close(dq, qt.grad.numpy())
+        close(dk, kt.grad.numpy())
+        close(dv, vt.grad.numpy())
+
+
+def pin_varlen_backward_gqa_is_summed_mha():
+    """GQA gradients = MHA gradients on K/V repeated per q-head, with dK and dV
+    summed over each group's heads."""
+    h_q, h_kv, d, scale = 6, 2, 4, 0.5
+    cq, ck, q, k, v, do = _varlen_case(18, [7, 4], [7, 4], h_q, h_kv, d)
+    G = h_q // h_kv
+    dq, dk, dv = oracle.varlen_backward(q, k, v, do, cq, ck, h_q, h_kv, True, scale)
+    dq2, dk2, dv2 = oracle.varlen_backward(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1), do, cq, ck,
+                                           h_q, h_q, True, scale)
+    close(dq, dq2)
+    close(dk, dk2.reshape(dk2.shape[0], h_kv, G, d).sum(axis=2))
+    close(dv, dv2.reshape(dv2.shape[0], h_kv, G, d).sum(axis=2))
+
+
+def pin_varlen_backward_finite_differences():
+    """Central differences of sum dO . O (O from the oracle's masked softmax)."""
+    h_q, h_kv, d, scale, eps = 2, 1, 5, 0.6, 1e-5
+    cq, ck, q, k, v, do = _varlen_case(19, [6], [8], h_q, h_kv, d)
+    allowed = A.allowed_mask(6, 8, True)
+
+    def loss(q, k, v):
+        tot = 0.0
+        for hq in range(h_q):
+            O, _, _ = oracle.softmax_over_kept(scale * (q[:, hq] @ k[:, 0].T), allowed, v[:, 0])
+            tot += float((do[:, hq] * O).sum())
+        return tot
+
+    dq, dk, dv = oracle.varlen_backward(q, k, v, do, cq, ck, h_q, h_kv, True, scale)
+    rng = np.random.default_rng(20)
+    for which, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(5):
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += eps
+            minus[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            fd = (loss(**{**args, which: plus}) - loss(**{**args, which: minus})) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), (which, idx, fd, grad[idx])
+
+
+def pin_varlen_backward_dead_rows():
+    """Causal with s_q > s_k: the first s_q - s_k rows see no key, so their dQ
+    is zero and they add nothing to dK or dV; an empty sequence gives zeros."""
+    h_q, h_kv, d = 2, 2, 4
+    cq, ck, q, k, v, do = _varlen_case(21, [6, 0], [2, 3], h_q, h_kv, d)
+    dq, dk, dv = oracle.varlen_backward(q, k, v, do, cq, ck, h_q, h_kv, True, 0.5)
+    close(dq[:4], np.zeros_like(dq[:4]))
+    dq2, dk2, dv2 = oracle.varlen_backward(q[4:6], k[:2], v[:2], do[4:6], [0, 2], [0, 2], h_q, h_kv, True, 0.5)
+    close(dk[:2], dk2)
+    close(dv[:2], dv2)
+    close(dq[4:6], dq2)
+    close(dk[2:], np.zeros_like(dk[2:]))
+
 ALL_PINS = [
     pin_bf16_codec, pin_two_by_two, pin_causal_two_by_two, pin_single_key, pin_uniform_scores,
     pin_dense_matches_sdpa, pin_gqa_equals_repeated_mha, pin_paged_equals_contiguous, pin_paged_prefill,
@@ -583,4 +681,6 @@ ALL_PINS = [
     pin_threshold_zero_is_dense, pin_threshold_one, pin_literal_equals_vectorised,
     pin_probabilities_sum_to_one, pin_smallseq_equals_varlen, pin_decode_skip_matches_literal,
     pin_smallseq_backward_autograd, pin_smallseq_backward_finite_differences, pin_smallseq_backward_single_key,
+    pin_varlen_backward_autograd, pin_varlen_backward_gqa_is_summed_mha, pin_varlen_backward_finite_differences,
+    pin_varlen_backward_dead_rows,
 ]

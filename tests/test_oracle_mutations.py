@@ -52,6 +52,11 @@ MUTANTS = [
     ("smallseq_backward", "scale * dS[:, None] * qf[b, hh][None, :]", "scale * dS[:, None] * of[b, hh][None, :]",
      "grad_K scales dO instead of q"),
     ("smallseq_backward", "P[:, None] * dO[None, :]", "P[::-1, None] * dO[None, :]", "grad_V keys reversed"),
+    ("varlen_backward", "dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))", "dS = P * dP",
+     "varlen softmax backward drops the row term"),
+    ("varlen_backward", "dk[k0:k1, hk] += scale * (dS.T @ Q)", "dk[k0:k1, hk] += dS.T @ Q", "dK without the scale"),
+    ("varlen_backward", "dv[k0:k1, hk] += P.T @ dO", "dv[k0:k1, hk] = P.T @ dO", "dV not summed over the group"),
+    ("varlen_backward", "dq[q0:q1, hq] = scale * (dS @ K)", "dq[q0:q1, hq] = scale * (dS @ V)", "dQ from V"),
     ("literal_group_attention", "acc[r][c] *= alpha", "acc[r][c] *= 1.0", "missing O rescale"),
     ("literal_group_attention", "l[r] *= alpha", "l[r] *= 1.0", "missing l rescale"),
     ("bf16_bits_to_f64", "<< 16", "<< 15", "bf16 decode shift"),
