@@ -43,6 +43,8 @@ EXPORTS = {
     "attn_paged_decode_workspace_size_ex": (_S, [_I, _I, _I, _I, _F]),
     "attn_smallseq_fwd": (_I, [_P] * 4 + [_I] * 5 + [_F, _P, _P, _P]),
     "attn_smallseq_bwd": (_I, [_P] * 6 + [_I] * 5 + [_F, _P, _P, _P, _P]),
+    "attn_varlen_bwd_workspace_size": (_S, [_I, _I]),
+    "attn_varlen_bwd": (_I, [_P] * 8 + [_I] * 9 + [_F] + [_P] * 4 + [_S, _P]),
     "attn_get_last_device_error": (_I, [_P]),
 }
 for _name, (_res, _args) in EXPORTS.items():
@@ -175,6 +177,35 @@ def prefill_skip_mask_words(batch, max_q, max_k, h_q, block_m=128, skip_tile=32)
     qb = -(-max_q // block_m)
     kt = -(-max_k // skip_tile)
     return -(-(batch * qb * h_q * kt) // 32), qb, kt
+
+
+def attn_varlen_bwd(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_q, max_k, causal=True, scale=None,
+                    dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of attn_varlen_fwd from its output and log-sum-exp.  dout like
+    out; returns (dq [Tq, h_q, d], dk, dv [Tk, h_kv, d])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 2)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, h_q, d = q.shape
+    total_k, h_kv, _ = k.shape
+    if dq is None:
+        dq = torch.empty_like(q)
+    if dk is None:
+        dk = torch.empty_like(k)
+    if dv is None:
+        dv = torch.empty_like(v)
+    need = int(lib.attn_varlen_bwd_workspace_size(total_q, h_q))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib.attn_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens_q),
+                             _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, total_q, total_k, int(max_q), int(max_k),
+                             h_q, h_kv, d, 1 if causal else 0, scale, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_varlen_bwd", rc)
+    return dq, dk, dv
 
 
 def attn_paged_decode_workspace_size(batch, h_q, d, max_pages_per_seq=0, skip_threshold=0.0):

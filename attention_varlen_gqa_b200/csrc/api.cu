@@ -196,6 +196,72 @@ int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *
   return launch_prefill(p, qmap, kmap, vmap, omap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
 }
 
+size_t attn_varlen_bwd_workspace_size(int total_q, int h_q) {
+  if (total_q <= 0 || h_q <= 0) return 256;
+  return align_up((size_t)total_q * h_q * sizeof(float), 256);
+}
+
+int attn_varlen_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v, const attn_bf16 *out,
+                    const attn_bf16 *dout, const float *lse, const int32_t *cu_seqlens_q,
+                    const int32_t *cu_seqlens_k, int batch, int total_q, int total_k, int max_q, int max_k,
+                    int h_q, int h_kv, int d, int causal, float scale, attn_bf16 *dq, attn_bf16 *dk,
+                    attn_bf16 *dv, void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  if (batch < 0 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0) return ATTN_E_SHAPE;
+  if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
+  if (batch > 0 && (max_q <= 0 || total_q <= 0)) return ATTN_E_SHAPE;
+  if (!q || !k || !v || !out || !dout || !lse || !cu_seqlens_q || !cu_seqlens_k || !dq || !dk || !dv)
+    return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_E_ALIGN;
+  if ((long long)max_q > (1ll << 24) || (long long)max_k > (1ll << 24)) return ATTN_E_TOO_LARGE;
+  if (batch > 0) {
+    if (!workspace) return ATTN_E_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_E_ALIGN;
+    if (workspace_bytes < attn_varlen_bwd_workspace_size(total_q, h_q)) return ATTN_E_WORKSPACE;
+  }
+  unsigned int *err = nullptr;
+  int rc = device_state(&err);
+  if (rc) return rc;
+  if (batch == 0) return ATTN_OK;
+  BwdParams p{};
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.delta = static_cast<float *>(workspace);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.batch = batch;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.max_q = max_q;
+  p.max_k = max_k;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.group = h_q / h_kv;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.qb_max = (max_q + kPrefillBlockM - 1) / kPrefillBlockM;
+  p.kt_max = (max_k + kPrefillBlockN - 1) / kPrefillBlockN;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err;
+  CUtensorMap qmap, kmap, vmap, dmap;
+  if (encode_3d(&qmap, q, d, h_q, total_q, kPrefillBlockM) ||
+      encode_3d(&kmap, k, d, h_kv, total_k, kPrefillBlockN) ||
+      encode_3d(&vmap, v, d, h_kv, total_k, kPrefillBlockN) ||
+      encode_3d(&dmap, dout, d, h_q, total_q, kPrefillBlockM))
+    return ATTN_E_CUDA;
+  return launch_backward(p, qmap, kmap, vmap, dmap, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? ATTN_OK
+             : ATTN_E_CUDA;
+}
+
 int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
                        const int32_t *block_table, const int32_t *cu_seqlens_q, const int32_t *seq_lens_k,
                        int batch, int total_q, int max_q, int max_k, int num_pages, int max_pages_per_seq,

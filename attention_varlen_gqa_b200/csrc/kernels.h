@@ -29,6 +29,19 @@ struct SmallSeqParams {
   unsigned int *err;
 };
 
+struct BwdParams {
+  const int32_t *cu_q, *cu_k;
+  const uint16_t *out, *dout;   // [total_q, h_q, d] the forward's output and its gradient
+  const float *lse;             // [total_q, h_q] the forward's log-sum-exp (natural log)
+  float *delta;                 // [total_q, h_q] workspace: <dO, O> per row
+  uint16_t *dq;                 // [total_q, h_q, d]
+  uint16_t *dk, *dv;            // [total_k, h_kv, d]
+  int batch, total_q, total_k, max_q, max_k, h_q, h_kv, group, d, causal;
+  int qb_max, kt_max;           // ceil(max_q / 128), ceil(max_k / 128)
+  float scale, scale_log2;
+  unsigned int *err;
+};
+
 struct DecodeParams {
   const uint16_t *q;            // [B, h_q, d]
   const int32_t *block_table;   // [B, max_pages]
@@ -69,6 +82,8 @@ struct PrefillParams {
 };
 
 cudaError_t launch_smallseq(const SmallSeqParams &p, cudaStream_t stream);
+cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                            const CUtensorMap &vmap, const CUtensorMap &dmap, cudaStream_t stream);
 cudaError_t launch_smallseq_bwd(const SmallSeqParams &p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);

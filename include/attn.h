@@ -7,7 +7,8 @@
  *   attn_varlen_fwd     packed variable-length GQA prefill, causal or not
  *                       (NVIDIA/Model-Optimizer PR 1034, "Add Triton unified
  *                       attention kernel with HuggingFace integration":
- *                       variable-length batching, GQA, causal/non-causal).
+ *                       variable-length batching, GQA, causal/non-causal),
+ *                       and attn_varlen_bwd, its gradients.
  *   attn_paged_decode   one query token per sequence against a paged KV cache
  *                       (NVIDIA/Model-Optimizer PR 1941, "Add split-k decode
  *                       kernel for skip softmax": a 32-split schedule of
@@ -212,6 +213,39 @@ ATTN_API int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, co
                        float skip_threshold, uint32_t *skip_mask,
                        unsigned long long *skip_counts,
                        attn_bf16 *out, float *lse, attn_stream_t stream);
+
+/*
+ * attn_varlen_bwd -- gradients of attn_varlen_fwd (skip threshold 0) with
+ * respect to q, k and v, for training through autograd (NVIDIA/Model-Optimizer
+ * PR 1034, "Add Triton unified attention kernel with HuggingFace
+ * integration", description).  With P = exp(scale * Q K^T - lse) over the
+ * allowed keys (the same masks as the forward), Delta_i = <dO_i, O_i>,
+ * dP = dO V^T and dS = P * (dP - Delta):
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO,
+ * dK and dV summed over the q-heads of each kv-head's group.
+ *
+ *   q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_q,
+ *   max_k, h_q, h_kv, d, causal, scale   as passed to attn_varlen_fwd
+ *   out            [total_q, h_q, d] bf16, the forward's output
+ *   dout           [total_q, h_q, d] bf16, the loss gradient w.r.t. out
+ *   lse            [total_q, h_q] float32, the forward's log-sum-exp (natural
+ *                  log, -inf for rows with no key)
+ *   dq             [total_q, h_q, d] bf16 output
+ *   dk, dv         [total_k, h_kv, d] bf16 outputs; every key of a valid
+ *                  sequence is written (zero when no query sees it)
+ *   workspace      device buffer of >= attn_varlen_bwd_workspace_size(total_q,
+ *                  h_q) bytes, 16-byte aligned (Delta per row); required
+ *                  when batch > 0
+ * A sequence with an invalid cu_seqlens range sets ATTN_DEVERR_CU_SEQLENS and
+ * none of its rows are written.  The result is deterministic (no atomics).
+ */
+ATTN_API size_t attn_varlen_bwd_workspace_size(int total_q, int h_q);
+ATTN_API int attn_varlen_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v,
+                             const attn_bf16 *out, const attn_bf16 *dout, const float *lse,
+                             const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int batch,
+                             int total_q, int total_k, int max_q, int max_k, int h_q, int h_kv, int d,
+                             int causal, float scale, attn_bf16 *dq, attn_bf16 *dk, attn_bf16 *dv,
+                             void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * attn_paged_decode_workspace_size -- bytes of workspace attn_paged_decode

@@ -196,3 +196,29 @@ def test_smallseq_bwd_argument_errors(A):
     assert smallseq_bwd(A, w=FAKE + 1) == -2
     assert smallseq_bwd(A, dq=FAKE + 8) == -2
     assert smallseq_bwd(A, scale=0.0) == -10
+
+
+def varlen_bwd(A, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, do=FAKE, lse=FAKE, cq=FAKE, ck=FAKE, batch=2, tq=10, tk=10, mq=5, mk=5,
+             hq=4, hkv=2, d=64, causal=1, scale=0.125, dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return A.lib.attn_varlen_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["cq"], a["ck"], a["batch"],
+                                 a["tq"], a["tk"], a["mq"], a["mk"], a["hq"], a["hkv"], a["d"], a["causal"],
+                                 a["scale"], a["dq"], a["dk"], a["dv"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_varlen_bwd_argument_errors(A):
+    assert varlen_bwd(A, hq=3) == -3
+    assert varlen_bwd(A, d=96) == -4
+    assert varlen_bwd(A, scale=0.0) == -10
+    assert varlen_bwd(A, batch=-1) == -8
+    assert varlen_bwd(A, lse=None) == -1
+    assert varlen_bwd(A, do=None) == -1
+    assert varlen_bwd(A, dk=None) == -1
+    assert varlen_bwd(A, dq=FAKE + 8) == -2
+    assert varlen_bwd(A, lse=FAKE + 2) == -2
+    assert varlen_bwd(A, ws=None) == -9
+    assert varlen_bwd(A, wsb=8) == -9
+    assert varlen_bwd(A, mk=1 << 25) == -13
+    assert A.lib.attn_varlen_bwd_workspace_size(10, 4) == 256
+    assert A.lib.attn_varlen_bwd_workspace_size(1000, 32) == 1000 * 32 * 4

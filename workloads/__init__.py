@@ -330,3 +330,9 @@ def smallseq_grad_inputs(s, seed=0, where="host"):
     tot = u.sum(dim=3, keepdim=True)
     w = torch.where(tot > 0, u / tot.clamp_min(1e-30), torch.zeros_like(u))
     return dict(dout=dout, weights=w.to(torch.bfloat16))
+
+
+def output_grad(data, seed=0, where="host"):
+    """dO ~ N(0, 1) (bf16) shaped like the query tensor of a prefill case."""
+    shape = (int(data["cu_seqlens_q"][-1]), data["h_q"], data["d"])
+    return _values(np.random.default_rng(seed + 104729), shape, where, seed, 6)
