@@ -113,12 +113,6 @@ ATTN_DEVICE Seq seq_at(const BwdParams &p, int b) {
   return s;
 }
 
-// Key j may be seen by query i (both local to the sequence): bottom-right
-// aligned causal mask, varlen bounds.
-ATTN_DEVICE bool allowed(const BwdParams &p, const Seq &s, int i, int j) {
-  return i < s.s_q && j < s.s_k && (!p.causal || j <= i + (s.s_k - s.s_q));
-}
-
 // Query blocks [r0, r1) of a sequence that see key tile t.
 ATTN_DEVICE void blocks_seeing(const BwdParams &p, const Seq &s, int t, int &r0, int &r1) {
   r1 = (s.s_q + BT - 1) / BT;
@@ -345,6 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int r = r0 + it % per_head;
       const float *lv = vec + st * 2 * BT;
+      // this key may be seen by the block's queries (columns) [lo, hi)
+      const int hi = j < s.s_k ? min(BT, s.s_q - r * BT) : 0;
+      const int lo = p.causal ? max(0, j - (s.s_k - s.s_q) - r * BT) : 0;
+      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == BT);
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * wg + cc;                    // 32 queries [32 c, 32 c + 32) of the block
@@ -360,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int col = 32 * c + e + u;
-            const bool a = allowed(p, s, r * BT + col, j);
-            pv[u] = a ? ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lv[col])) : 0.f;
+            const float x = ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lv[col]));
+            pv[u] = (full || (col >= lo && col < hi)) ? x : 0.f;
             dv[u] = pv[u] * (__uint_as_float(dr[e + u]) - lv[BT + col]);
           }
           pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
@@ -586,11 +584,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t vrow = (size_t)(s.q0 + (in ? i : 0)) * p.h_q + hq;
     const float lse2 = in ? __ldg(p.lse + vrow) * kLog2e : 0.f;
     const float delta = in ? __ldg(p.delta + vrow) : 0.f;
+    // this query sees the keys [0, k_lim) of its sequence
+    const int k_lim = in ? (p.causal ? min(s.s_k, i + (s.s_k - s.s_q) + 1) : s.s_k) : 0;
     bool ok = true;
     for (int jt = 0; jt < nt && ok; ++jt) {
       ok = __all_sync(0xffffffffu, wait_bar(sd_full, jt & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
+      const int lim = k_lim - jt * BT;                 // allowed columns of this tile: [0, lim)
+      const bool full = __all_sync(0xffffffffu, lim >= BT);
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * wg + cc;                    // keys [32 c, 32 c + 32) of the tile
@@ -605,8 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const bool a = allowed(p, s, i, jt * BT + 32 * c + e + u);
-            const float pv = a ? ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lse2)) : 0.f;
+            const float x = ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lse2));
+            const float pv = (full || 32 * c + e + u < lim) ? x : 0.f;
             dv[u] = pv * (__uint_as_float(dr[e + u]) - delta);
           }
           dk[e / 2] = pack_bf16x2(dv[0], dv[1]);

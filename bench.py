@@ -52,11 +52,11 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip", "smallseq_bwd",
-                                       "decode_skip"],
+                                       "decode_skip", "varlen_bwd"],
                     default="all",
                     help="profiling aid: run a single operation (no JSON line)")
     ap.add_argument("--no-skip", action="store_true",
-                    help="leave out the skip-softmax, paged-prefill and small-seq backward measurements")
+                    help="leave out the skip-softmax, paged-prefill and the two backward measurements")
     ap.add_argument("--no-cpu", action="store_true", help="leave out the CPU oracle baseline")
     ap.add_argument("--small", action="store_true",
                     help="profiling aid with --only: quarter-size decode / small-seq batches")
@@ -350,6 +350,10 @@ def main():
     if args.only == "skip":
         measure_skip(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
         return
+    if args.only == "varlen_bwd":
+        measure_varlen_bwd(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
+        assert A.attn_get_last_device_error() == 0
+        return
     if args.only == "smallseq_bwd":
         measure_smallseq_bwd(A, W, torch, dev, seed, pk, reps=max(1, args.steps),
                              batch=7680 if args.small else 30720)
@@ -428,11 +432,12 @@ def main():
     agg = aggregate_ranks({"per": per, "total_ms": total_ms, "e2e_ms": e2e_ms_local, "flops": pre_flops,
                            "dec_bytes": dec_bytes, "ss_bytes": ss_bytes}, world, dev)
 
-    skip = paged = ssb = None
+    skip = paged = ssb = vbwd = None
     if not args.no_skip:
         skip = measure_skip(A, W, torch, dev, seed, pk, reps=3)
         paged = measure_paged_prefill(A, W, torch, dev, seed, pk, reps=3)
         ssb = measure_smallseq_bwd(A, W, torch, dev, seed, pk, reps=5)
+        vbwd = measure_varlen_bwd(A, W, torch, dev, seed, pk, reps=5)
 
     if rank != 0:
         if world > 1:
@@ -481,6 +486,7 @@ def main():
         "skip": skip,
         "paged_prefill": paged,
         "smallseq_bwd": ssb,
+        "varlen_bwd": vbwd,
         "cpu_baseline": cpu,
         "e2e": {"value": agg["e2e_value"], "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": agg["e2e_ms"],
@@ -599,6 +605,40 @@ def measure_paged_prefill(A, W, torch, dev, seed, pk, reps=3):
                         "h 32/8, d 128, page 16, causal",
             "ms": ms, "flops": flops, "tflops": flops / ms / 1e9, "frac_of_measured": flops / ms / 1e9 / pk["bf16"],
             "lens_k": [int(x) for x in lens_k]}
+
+
+def measure_varlen_bwd(A, W, torch, dev, seed, pk, reps=5):
+    """Varlen GQA backward on the prefill workload (8 sequences, 24 900 tokens,
+    h 32/8, d 128, causal) from the GPU forward's output and LSE, dO ~ N(0, 1).
+    FLOPs: 2.5 x the forward's (the five matrix products of the backward: S,
+    dP, dV, dK, dQ); the kernels recompute S and dP once more.  Not a step
+    row: reported beside it."""
+    w = W.gqa_prefill(seed=seed, where="device")
+    dout = W.output_grad(w, seed=seed, where="device")
+    cq = torch.from_numpy(w["cu_seqlens_q"]).to(dev)
+    ck = torch.from_numpy(w["cu_seqlens_k"]).to(dev)
+    o, lse = A.attn_varlen_fwd(w["q"], w["k"], w["v"], cq, ck, w["max_q"], w["max_k"], causal=True)
+    dq, dk, dv = torch.empty_like(w["q"]), torch.empty_like(w["k"]), torch.empty_like(w["v"])
+    ws = torch.empty(A.lib.attn_varlen_bwd_workspace_size(w["q"].shape[0], 32), dtype=torch.uint8, device=dev)
+
+    def run():
+        A.attn_varlen_bwd(w["q"], w["k"], w["v"], o, dout, lse, cq, ck, w["max_q"], w["max_k"], causal=True,
+                          dq=dq, dk=dk, dv=dv, workspace=ws)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    flops = 2.5 * prefill_flops(w["lens_q"], w["lens_k"], 32, 128, True)
+    tf = flops / ms / 1e9
+    return {"workload": "8 sequences U[512, 8192] seed 0 (24 900 tokens), h 32/8, d 128, causal; dO ~ N(0, 1)",
+            "ms": ms, "flops": flops, "tflops": tf, "frac_of_measured": tf / pk["bf16"],
+            "frac_of_2250": tf / 2250.0}
 
 
 def measure_smallseq_bwd(A, W, torch, dev, seed, pk, reps=5, batch=30720):
