@@ -40,7 +40,7 @@ namespace {
 constexpr int BT = 128;                      // keys per tile, queries per block
 constexpr int kQStages = 2;                  // dK/dV kernel: query blocks in flight
 constexpr int kKVStages = 2;                 // dQ kernel: key tiles in flight
-constexpr int kEwWarps = 8;                  // two elementwise warpgroups
+constexpr int kEwWarps = 16;                 // four elementwise warpgroups, 32 columns each
 constexpr int kProducerWarp = kEwWarps;
 constexpr int kMmaWarp = kEwWarps + 1;
 constexpr int kThreads = 32 * (kEwWarps + 2);
@@ -309,12 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bDO = smem_desc_sw128(sDO, BT * 128, 1024), bQ = smem_desc_sw128(sQ, BT * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t a = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;    // P^T of queries [16 kk, 16 kk + 16)
+          const uint32_t a = 32 * (kk >> 1) + 8 * (kk & 1);    // P^T of queries [16 kk, 16 kk + 16)
           mma_ts(tmem + 256, tmem + a, bDO + ((kk * 16 * 128) >> 4), idPV, (it > 0 || kk > 0) ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t a = 128 + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);   // dS^T
+          const uint32_t a = 128 + 32 * (kk >> 1) + 8 * (kk & 1);   // dS^T
           mma_ts(tmem + 384, tmem + a, bQ + ((kk * 16 * 128) >> 4), idPV, (it > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&q_empty[st]);
@@ -342,31 +342,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this key may be seen by the block's queries (columns) [lo, hi)
       const int hi = j < s.s_k ? min(BT, s.s_q - r * BT) : 0;
       const int lo = p.causal ? max(0, j - (s.s_k - s.s_q) - r * BT) : 0;
-      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == BT);
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * wg + cc;                    // 32 queries [32 c, 32 c + 32) of the block
+      const int c = wg;                               // 32 queries [32 c, 32 c + 32) of the block
+      const bool full = __all_sync(0xffffffffu, lo <= 32 * c && hi >= 32 * c + 32);
+      {
         uint32_t sr[32], dr[32], pk[16], dk[16];
         tmem_ld32(tS + 32 * c, sr);
         tmem_ld32(tP + 32 * c, dr);
         tmem_wait_ld();
         tie(sr);
         tie(dr);
+        const float4 *l4 = reinterpret_cast<const float4 *>(lv + 32 * c);
+        const float4 *d4 = reinterpret_cast<const float4 *>(lv + BT + 32 * c);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], dv[2];
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 lq = l4[e4], dq = d4[e4];
+          const float la[4] = {lq.x, lq.y, lq.z, lq.w}, da[4] = {dq.x, dq.y, dq.z, dq.w};
+          float pv[4], dv[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 32 * c + e + u;
-            const float x = ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lv[col]));
+          for (int u = 0; u < 4; ++u) {
+            const int e = 4 * e4 + u, col = 32 * c + e;
+            const float x = ex2(fmaf(__uint_as_float(sr[e]), p.scale_log2, -la[u]));
             pv[u] = (full || (col >= lo && col < hi)) ? x : 0.f;
-            dv[u] = pv[u] * (__uint_as_float(dr[e + u]) - lv[BT + col]);
+            dv[u] = pv[u] * (__uint_as_float(dr[e]) - da[u]);
           }
-          pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
-          dk[e / 2] = pack_bf16x2(dv[0], dv[1]);
+          pk[2 * e4] = pack_bf16x2(pv[0], pv[1]);
+          pk[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[2 * e4] = pack_bf16x2(dv[0], dv[1]);
+          dk[2 * e4 + 1] = pack_bf16x2(dv[2], dv[3]);
         }
-        tmem_st16(tS + 64 * wg + 16 * cc, pk);        // P^T over S^T columns this warpgroup has read
-        tmem_st16(tP + 64 * wg + 16 * cc, dk);        // dS^T over dP^T columns
+        tmem_st16(tS + 32 * c, pk);                   // P^T over this warpgroup's own S^T columns
+        tmem_st16(tP + 32 * c, dk);                   // dS^T over its own dP^T columns
       }
       tmem_wait_st();
       tc_fence_before();
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tile's keys that belong to the sequence are stored
       const size_t out_row = ((size_t)(s.k0 + min(j, s.s_k - 1)) * p.h_kv + hk) * D;
 #pragma unroll 1
-      for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {   // 32-column chunks
+      for (int c = wg; c < D / 32; c += 4) {   // 32-column chunks of dV and dK
         uint32_t v[32], kv[32];
         if (have && ok) {
           tmem_ld32(tmem + lane_addr + 256 + 32 * c, v);
@@ -564,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bKmn = smem_desc_sw128(sK, BT * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t a = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;   // dS of keys [16 kk, 16 kk + 16)
+          const uint32_t a = 32 * (kk >> 1) + 8 * (kk & 1);   // dS of keys [16 kk, 16 kk + 16)
           mma_ts(tmem + 256, tmem + a, bKmn + ((kk * 16 * 128) >> 4), idPV, (jt > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&kv_empty[st]);
@@ -592,10 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int lim = k_lim - jt * BT;                 // allowed columns of this tile: [0, lim)
-      const bool full = __all_sync(0xffffffffu, lim >= BT);
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * wg + cc;                    // keys [32 c, 32 c + 32) of the tile
+      const int c = wg;                               // keys [32 c, 32 c + 32) of the tile
+      const bool full = __all_sync(0xffffffffu, lim >= 32 * c + 32);
+      {
         uint32_t sr[32], dr[32], dk[16];
         tmem_ld32(tS + 32 * c, sr);
         tmem_ld32(tP + 32 * c, dr);
@@ -613,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           dk[e / 2] = pack_bf16x2(dv[0], dv[1]);
         }
-        tmem_st16(tS + 64 * wg + 16 * cc, dk);        // dS over S columns this warpgroup has read
+        tmem_st16(tS + 32 * c, dk);                   // dS over this warpgroup's own S columns
       }
       tmem_wait_st();
       tc_fence_before();
@@ -629,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warp-wide TMEM loads by every lane; rows of the sequence are stored
       const size_t out_row = ((size_t)(s.q0 + (in ? i : 0)) * p.h_q + hq) * D;
 #pragma unroll 1
-      for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
+      for (int c = wg; c < D / 32; c += 4) {
         uint32_t v[32];
         if (have && ok) {
           tmem_ld32(tmem + lane_addr + 256 + 32 * c, v);
