@@ -217,6 +217,10 @@ int attn_varlen_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *v, 
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_E_ALIGN;
   if ((long long)max_q > (1ll << 24) || (long long)max_k > (1ll << 24)) return ATTN_E_TOO_LARGE;
+  // one CTA per (query block or key tile, head, sequence): the grids must fit 2^31 - 1
+  if ((long long)batch * h_q * ((max_q + kPrefillBlockM - 1) / kPrefillBlockM) >= (1ll << 31) ||
+      (long long)batch * h_kv * ((max_k + kPrefillBlockN - 1) / kPrefillBlockN) >= (1ll << 31))
+    return ATTN_E_TOO_LARGE;
   if (batch > 0) {
     if (!workspace) return ATTN_E_WORKSPACE;
     if (!aligned16(workspace)) return ATTN_E_ALIGN;

@@ -199,7 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *vec = reinterpret_cast<float *>(sm + L::kVec);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hk = blockIdx.x % p.h_kv, b = blockIdx.x / p.h_kv, t = blockIdx.y;
+  // the key tiles of one (sequence, kv-head) are neighbours in launch order,
+  // so they run together and read its query blocks while those sit in L2
+  const int t = (int)(blockIdx.x % (unsigned)p.kt_max);
+  const int grp = (int)(blockIdx.x / (unsigned)p.kt_max);
+  const int hk = grp % p.h_kv, b = grp / p.h_kv;
   const int G = p.group;
   const Seq s = seq_at(p, b);
   if (s.bad || t * BT >= s.s_k) return;       // the whole CTA leaves before any barrier
@@ -464,12 +468,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hq = blockIdx.x % p.h_q, b = blockIdx.x / p.h_q;
-  const int r = p.qb_max - 1 - (int)blockIdx.y;   // the heaviest (last) causal blocks first
+  // (sequence, q-head) fastest; the heaviest (last) causal query blocks first
+  const int bh = (int)(blockIdx.x % (unsigned)(p.batch * p.h_q));
+  const int r = p.qb_max - 1 - (int)(blockIdx.x / (unsigned)(p.batch * p.h_q));
+  const int hq = bh % p.h_q, b = bh / p.h_q;
   const int hk = hq / p.group;
   const Seq s = seq_at(p, b);
   if (s.bad) {
-    if (threadIdx.x == 0 && blockIdx.y == 0 && hq == 0) raise_error(p.err, ATTN_DEVERR_CU_SEQLENS);
+    if (threadIdx.x == 0 && r == p.qb_max - 1 && hq == 0) raise_error(p.err, ATTN_DEVERR_CU_SEQLENS);
     return;
   }
   if (r * BT >= s.s_q) return;
@@ -689,10 +695,9 @@ cudaError_t launch_bwd_d(const BwdParams &p, const CUtensorMap &qmap, const CUte
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, QLayout<D>::kBytes);
   if (e != cudaSuccess) return e;
-  // key tiles with the most query blocks (the first ones, causally) are launched first
-  bwd_dkdv_kernel<D><<<dim3(p.batch * p.h_kv, p.kt_max), kThreads, KvLayout<D>::kBytes, stream>>>(
+  bwd_dkdv_kernel<D><<<(unsigned)p.kt_max * p.batch * p.h_kv, kThreads, KvLayout<D>::kBytes, stream>>>(
       qmap, kmap, vmap, dmap, p);
-  bwd_dq_kernel<D><<<dim3(p.batch * p.h_q, p.qb_max), kThreads, QLayout<D>::kBytes, stream>>>(
+  bwd_dq_kernel<D><<<(unsigned)p.batch * p.h_q * p.qb_max, kThreads, QLayout<D>::kBytes, stream>>>(
       qmap, kmap, vmap, dmap, p);
   return cudaGetLastError();
 }
