@@ -175,8 +175,8 @@ struct KvLayout {
   static constexpr int kDO = kQ + kQStages * kTile;     // [stage] its output gradient
   static constexpr int kVec = kDO + kQStages * kTile;   // [stage] L * log2(e) [128], Delta [128]
   static constexpr int kBar = kVec + kQStages * BT * 2 * 4;
-  // kv_full, q_full[S], q_empty[S], sd_full, p_ready, done
-  static constexpr int kNumBars = 4 + 2 * kQStages;
+  // kv_full, q_full[S], q_empty[S], s_full, dp_full, p_done, ds_done, done
+  static constexpr int kNumBars = 6 + 2 * kQStages;
   static constexpr int kMisc = kBar + kNumBars * 8;     // TMEM address, abort flag
   // at least ~116 KB, so that one CTA (and its 512 TMEM columns) owns an SM
   static constexpr int kBytes = (kMisc + 16 + 1024 > 118 * 1024) ? kMisc + 16 + 1024 : 118 * 1024;
@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sm = align1024(smem_raw);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBar);
   uint64_t *kv_full = bars, *q_full = bars + 1, *q_empty = q_full + kQStages;
-  uint64_t *sd_full = q_empty + kQStages, *p_ready = sd_full + 1, *done = p_ready + 1;
+  uint64_t *s_full = q_empty + kQStages, *dp_full = s_full + 1, *p_done = dp_full + 1, *ds_done = p_done + 1;
+  uint64_t *done = ds_done + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::kMisc + 4);
   float *vec = reinterpret_cast<float *>(sm + L::kVec);
@@ -218,8 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[st], 1);
       mbar_init(&q_empty[st], 1);
     }
-    mbar_init(sd_full, 1);
-    mbar_init(p_ready, kEwWarps);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_done, kEwWarps);
+    mbar_init(ds_done, kEwWarps);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -299,23 +302,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem, dK0 + kmajor_step<D>(kk), dQ + kmajor_step<D>(kk), idS, kk > 0 ? 1u : 0u);
+        tc_commit(s_full);     // the elementwise warps start on P^T while dP^T runs
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + 128, dV0 + kmajor_step<D>(kk), dDO + kmajor_step<D>(kk), idS, kk > 0 ? 1u : 0u);
-        tc_commit(sd_full);
+        tc_commit(dp_full);
       }
       __syncwarp();
-      ok = __all_sync(0xffffffffu, wait_bar(p_ready, it & 1, abort_flag, p.err));
+      ok = __all_sync(0xffffffffu, wait_bar(p_done, it & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
+      // B operands MN-major: rows = queries (K), 64-column halves of D (N)
+      const uint64_t bDO = smem_desc_sw128(sDO, BT * 128, 1024), bQ = smem_desc_sw128(sQ, BT * 128, 1024);
       if (leader) {
-        // B operands MN-major: rows = queries (K), 64-column halves of D (N)
-        const uint64_t bDO = smem_desc_sw128(sDO, BT * 128, 1024), bQ = smem_desc_sw128(sQ, BT * 128, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk) {
+        for (int kk = 0; kk < BT / 16; ++kk) {   // dV while the elementwise warps form dS^T
           const uint32_t a = 32 * (kk >> 1) + 8 * (kk & 1);    // P^T of queries [16 kk, 16 kk + 16)
           mma_ts(tmem + 256, tmem + a, bDO + ((kk * 16 * 128) >> 4), idPV, (it > 0 || kk > 0) ? 1u : 0u);
         }
+      }
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, wait_bar(ds_done, it & 1, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
           const uint32_t a = 128 + 32 * (kk >> 1) + 8 * (kk & 1);   // dS^T
@@ -338,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < nb && ok; ++it) {
       const int st = it % kQStages;
       ok = __all_sync(0xffffffffu, wait_bar(&q_full[st], (it / kQStages) & 1, abort_flag, p.err) &&
-                                       wait_bar(sd_full, it & 1, abort_flag, p.err));
+                                       wait_bar(s_full, it & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
       const int r = r0 + it % per_head;
@@ -349,38 +359,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c = wg;                               // 32 queries [32 c, 32 c + 32) of the block
       const bool full = __all_sync(0xffffffffu, lo <= 32 * c && hi >= 32 * c + 32);
       {
-        uint32_t sr[32], dr[32], pk[16], dk[16];
+        // P^T (while the dP^T product runs), handed over for dV; then dS^T
+        uint32_t sr[32], pk[16];
+        float pv[32];
         tmem_ld32(tS + 32 * c, sr);
-        tmem_ld32(tP + 32 * c, dr);
         tmem_wait_ld();
         tie(sr);
-        tie(dr);
         const float4 *l4 = reinterpret_cast<const float4 *>(lv + 32 * c);
-        const float4 *d4 = reinterpret_cast<const float4 *>(lv + BT + 32 * c);
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 lq = l4[e4], dq = d4[e4];
-          const float la[4] = {lq.x, lq.y, lq.z, lq.w}, da[4] = {dq.x, dq.y, dq.z, dq.w};
-          float pv[4], dv[4];
+          const float4 lq = l4[e4];
+          const float la[4] = {lq.x, lq.y, lq.z, lq.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int e = 4 * e4 + u, col = 32 * c + e;
             const float x = ex2(fmaf(__uint_as_float(sr[e]), p.scale_log2, -la[u]));
-            pv[u] = (full || (col >= lo && col < hi)) ? x : 0.f;
-            dv[u] = pv[u] * (__uint_as_float(dr[e]) - da[u]);
+            pv[e] = (full || (col >= lo && col < hi)) ? x : 0.f;
           }
-          pk[2 * e4] = pack_bf16x2(pv[0], pv[1]);
-          pk[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          pk[2 * e4] = pack_bf16x2(pv[4 * e4], pv[4 * e4 + 1]);
+          pk[2 * e4 + 1] = pack_bf16x2(pv[4 * e4 + 2], pv[4 * e4 + 3]);
+        }
+        tmem_st16(tS + 32 * c, pk);                   // P^T over this warpgroup's own S^T columns
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_done);
+        ok = __all_sync(0xffffffffu, wait_bar(dp_full, it & 1, abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t dr[32], dk[16];
+        tmem_ld32(tP + 32 * c, dr);
+        tmem_wait_ld();
+        tie(dr);
+        const float4 *d4 = reinterpret_cast<const float4 *>(lv + BT + 32 * c);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 dq = d4[e4];
+          const float da[4] = {dq.x, dq.y, dq.z, dq.w};
+          float dv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dv[u] = pv[4 * e4 + u] * (__uint_as_float(dr[4 * e4 + u]) - da[u]);
           dk[2 * e4] = pack_bf16x2(dv[0], dv[1]);
           dk[2 * e4 + 1] = pack_bf16x2(dv[2], dv[3]);
         }
-        tmem_st16(tS + 32 * c, pk);                   // P^T over this warpgroup's own S^T columns
         tmem_st16(tP + 32 * c, dk);                   // dS^T over its own dP^T columns
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
+      if (lane == 0) mbar_arrive(ds_done);
     }
     // epilogue: this warpgroup's half of the D columns of dV and dK
     const bool have = nb > 0;
@@ -446,8 +473,8 @@ struct QLayout {
   static constexpr int kK = kDO + kTile;                // [stage] key tile
   static constexpr int kV = kK + kKVStages * kTile;     // [stage] value tile
   static constexpr int kBar = kV + kKVStages * kTile;
-  // q_full, kv_full[S], kv_empty[S], sd_full, p_ready, done
-  static constexpr int kNumBars = 4 + 2 * kKVStages;
+  // q_full, kv_full[S], kv_empty[S], s_full, dp_full, ds_done, done
+  static constexpr int kNumBars = 5 + 2 * kKVStages;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = (kMisc + 16 + 1024 > 118 * 1024) ? kMisc + 16 + 1024 : 118 * 1024;
   static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
@@ -463,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sm = align1024(smem_raw);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBar);
   uint64_t *q_full = bars, *kv_full = bars + 1, *kv_empty = kv_full + kKVStages;
-  uint64_t *sd_full = kv_empty + kKVStages, *p_ready = sd_full + 1, *done = p_ready + 1;
+  uint64_t *s_full = kv_empty + kKVStages, *dp_full = s_full + 1, *ds_done = dp_full + 1, *done = ds_done + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::kMisc + 4);
 
@@ -487,8 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&kv_full[st], 1);
       mbar_init(&kv_empty[st], 1);
     }
-    mbar_init(sd_full, 1);
-    mbar_init(p_ready, kEwWarps);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_done, kEwWarps);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -561,13 +589,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem, aQ + kmajor_step<D>(kk), bK + kmajor_step<D>(kk), idS, kk > 0 ? 1u : 0u);
+        tc_commit(s_full);     // the elementwise warps form P while dP runs
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + 128, aDO + kmajor_step<D>(kk), bV + kmajor_step<D>(kk), idS, kk > 0 ? 1u : 0u);
-        tc_commit(sd_full);
+        tc_commit(dp_full);
       }
       __syncwarp();
-      ok = __all_sync(0xffffffffu, wait_bar(p_ready, jt & 1, abort_flag, p.err));
+      ok = __all_sync(0xffffffffu, wait_bar(ds_done, jt & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
       if (leader) {
@@ -599,36 +628,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k_lim = in ? (p.causal ? min(s.s_k, i + (s.s_k - s.s_q) + 1) : s.s_k) : 0;
     bool ok = true;
     for (int jt = 0; jt < nt && ok; ++jt) {
-      ok = __all_sync(0xffffffffu, wait_bar(sd_full, jt & 1, abort_flag, p.err));
+      ok = __all_sync(0xffffffffu, wait_bar(s_full, jt & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
       const int lim = k_lim - jt * BT;                 // allowed columns of this tile: [0, lim)
       const int c = wg;                               // keys [32 c, 32 c + 32) of the tile
       const bool full = __all_sync(0xffffffffu, lim >= 32 * c + 32);
       {
+        // P while the dP product runs, then dS
         uint32_t sr[32], dr[32], dk[16];
+        float pv[32];
         tmem_ld32(tS + 32 * c, sr);
-        tmem_ld32(tP + 32 * c, dr);
         tmem_wait_ld();
         tie(sr);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = ex2(fmaf(__uint_as_float(sr[e]), p.scale_log2, -lse2));
+          pv[e] = (full || 32 * c + e < lim) ? x : 0.f;
+        }
+        ok = __all_sync(0xffffffffu, wait_bar(dp_full, jt & 1, abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld32(tP + 32 * c, dr);
+        tmem_wait_ld();
         tie(dr);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float dv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const float x = ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lse2));
-            const float pv = (full || 32 * c + e + u < lim) ? x : 0.f;
-            dv[u] = pv * (__uint_as_float(dr[e + u]) - delta);
-          }
-          dk[e / 2] = pack_bf16x2(dv[0], dv[1]);
-        }
+        for (int e = 0; e < 32; e += 2)
+          dk[e / 2] = pack_bf16x2(pv[e] * (__uint_as_float(dr[e]) - delta),
+                                  pv[e + 1] * (__uint_as_float(dr[e + 1]) - delta));
         tmem_st16(tS + 32 * c, dk);                   // dS over this warpgroup's own S columns
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
+      if (lane == 0) mbar_arrive(ds_done);
     }
     const bool have = nt > 0;
     if (have) {
