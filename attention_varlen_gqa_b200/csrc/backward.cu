@@ -26,8 +26,8 @@
 // S and dP are computed twice (once per kernel): two more tensor-core passes
 // than a single kernel that adds dQ with atomics, no atomic traffic.
 // TMEM (512 columns): dK/dV kernel S^T [0,128) -> P^T, dP^T [128,256) ->
-// dS^T, dV [256,256+d), dK [384,384+d); dQ kernel S [0,128) -> dS, dP
-// [128,256), dQ [256,256+d).
+// dS^T, dV [256,256+d), dK [384,384+d); dQ kernel S [0,128), dP [128,256)
+// -> dS, dQ [256,256+d).
 #include <math.h>
 
 #include "common.cuh"
@@ -578,38 +578,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = nt > 0 && __all_sync(0xffffffffu, wait_bar(q_full, 0, abort_flag, p.err));
     const uint64_t aQ = smem_desc_sw128(sbase + L::kQ, 16, 1024);
     const uint64_t aDO = smem_desc_sw128(sbase + L::kDO, 16, 1024);
-    for (int jt = 0; jt < nt && ok; ++jt) {
-      const int st = jt % kKVStages;
-      ok = __all_sync(0xffffffffu, wait_bar(&kv_full[st], (jt / kKVStages) & 1, abort_flag, p.err));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t sK = sbase + L::kK + st * L::kTile, sV = sbase + L::kV + st * L::kTile;
+    // S of tile jt into columns [0, 128), its dP into [128, 256)
+    auto issue_s = [&](int jt) {
       if (leader) {
-        const uint64_t bK = smem_desc_sw128(sK, 16, 1024), bV = smem_desc_sw128(sV, 16, 1024);
+        const uint64_t bK = smem_desc_sw128(sbase + L::kK + (jt % kKVStages) * L::kTile, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem, aQ + kmajor_step<D>(kk), bK + kmajor_step<D>(kk), idS, kk > 0 ? 1u : 0u);
-        tc_commit(s_full);     // the elementwise warps form P while dP runs
+        tc_commit(s_full);
+      }
+      __syncwarp();
+    };
+    auto issue_dp = [&](int jt) {
+      if (leader) {
+        const uint64_t bV = smem_desc_sw128(sbase + L::kV + (jt % kKVStages) * L::kTile, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + 128, aDO + kmajor_step<D>(kk), bV + kmajor_step<D>(kk), idS, kk > 0 ? 1u : 0u);
         tc_commit(dp_full);
       }
       __syncwarp();
+    };
+    // Per tile: S, dP (the elementwise warps form P while dP runs); once dS
+    // is written (over dP's columns) the next tile's S, then dQ, then the next
+    // dP, so the next exponentials overlap dQ and dP.
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&kv_full[0], 0, abort_flag, p.err));
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+      issue_dp(0);
+    }
+    for (int jt = 0; jt < nt && ok; ++jt) {
+      const int st = jt % kKVStages;
+      const uint32_t sK = sbase + L::kK + st * L::kTile;
       ok = __all_sync(0xffffffffu, wait_bar(ds_done, jt & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
+      const bool more = jt + 1 < nt;
+      if (more) {
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(&kv_full[(jt + 1) % kKVStages], ((jt + 1) / kKVStages) & 1, abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(jt + 1);
+      }
       if (leader) {
         // B = the key tile MN-major: rows = keys (K), 64-column halves of D (N)
         const uint64_t bKmn = smem_desc_sw128(sK, BT * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t a = 32 * (kk >> 1) + 8 * (kk & 1);   // dS of keys [16 kk, 16 kk + 16)
+          const uint32_t a = 128 + 32 * (kk >> 1) + 8 * (kk & 1);   // dS of keys [16 kk, 16 kk + 16)
           mma_ts(tmem + 256, tmem + a, bKmn + ((kk * 16 * 128) >> 4), idPV, (jt > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&kv_empty[st]);
       }
       __syncwarp();
+      if (more) issue_dp(jt + 1);
     }
     if (leader) tc_commit(done);
     __syncwarp();
@@ -656,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; e += 2)
           dk[e / 2] = pack_bf16x2(pv[e] * (__uint_as_float(dr[e]) - delta),
                                   pv[e + 1] * (__uint_as_float(dr[e + 1]) - delta));
-        tmem_st16(tS + 32 * c, dk);                   // dS over this warpgroup's own S columns
+        tmem_st16(tP + 32 * c, dk);                   // dS over this warpgroup's own dP columns
       }
       tmem_wait_st();
       tc_fence_before();
