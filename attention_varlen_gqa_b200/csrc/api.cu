@@ -177,6 +177,8 @@ int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const attn_bf16 *
   p.scale_log2 = scale * 1.4426950408889634f;
   p.thr_log2 = thr_to_log2(skip_threshold);
   p.err = err;
+  // keys beyond the queries (chunked prefill): a sequence's items together
+  p.seq_major = max_k > max_q ? 1 : 0;
 
   if (skip_mask) {
     const size_t bits = (size_t)batch * p.qb_max * h_q * p.kt_max;
@@ -312,6 +314,8 @@ int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_
   p.scale_log2 = scale * 1.4426950408889634f;
   p.thr_log2 = thr_to_log2(skip_threshold);
   p.err = err;
+  // keys beyond the queries (chunked prefill): a sequence's items together
+  p.seq_major = max_k > max_q ? 1 : 0;
   p.paged = 1;
   p.num_pages = num_pages;
   p.max_pages = max_pages_per_seq;

@@ -74,6 +74,10 @@ struct PrefillParams {
   float scale_log2, thr_log2;
   unsigned int *err;
   int work_slot;                // work-claim counter of this launch (set by launch_prefill)
+  // item order: 0 = query blocks outermost (heaviest causal block first, for
+  // s_q = s_k); 1 = sequences outermost (all items that read one sequence's
+  // K/V run together, for prefixes longer than the queries)
+  int seq_major;
   // paged K/V (chunked prefill): keys and values of sequence b live in the
   // pages block_table[b, :] of a [num_pages, 16, h_kv, d] cache, s_k =
   // seq_lens_k[b]; cu_k / total_k are unused then

@@ -30,6 +30,7 @@
 // Waiting warps sleep in mbarrier.try_wait instead of spinning: every SM
 // sub-partition hosts two softmax warps, and spinning waiters took issue
 // slots from the one computing exponentials.
+#include <limits.h>
 #include <math.h>
 
 #include <atomic>
@@ -50,6 +51,9 @@ constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kSchedWarp = kMmaWarp + 1;
 constexpr int kSchedDepth = 4;                 // work items claimed ahead
 constexpr int kSchedConsumers = 4 * kNQ + 2;   // warps that read each claimed item
+// Sequences ranked for the sequence-major item order (batches of up to
+// kRankMax sequences; larger batches keep their own order).
+constexpr int kRankMax = 32;
 // Work-claim counters, one pair (next item, CTAs done) per launch slot; the
 // last CTA of a launch puts its pair back to zero.  Launches take slots in
 // turn, so up to kWorkSlots prefill launches may run at the same time on a
@@ -140,25 +144,44 @@ ATTN_DEVICE int num_items(const PrefillParams &p) {
   return p.batch * ((p.qb_max + 1) / 2) * p.h_q;
 }
 
-// Items are ordered by decreasing q-block index, i.e. heaviest causal work first.
-ATTN_DEVICE Item item_at(const PrefillParams &p, int idx) {
+// With sequences outermost, batches of up to kRankMax sequences take them
+// longest first (the ranking is made by each CTA's scheduler warp).
+ATTN_DEVICE bool ranked(const PrefillParams &p) { return p.seq_major && p.batch <= kRankMax; }
+
+// Items are numbered heaviest first.  With seq_major == 0 the query-block
+// index (counted from the last block) is the outer digit, so every
+// sequence's last, causally heaviest, blocks come first; with seq_major == 1
+// the ranked sequence is the outer digit and the query block the next.  The
+// two query tiles of an item are two heads of one kv-head (even group), or
+// two query blocks of one head (odd group).
+ATTN_DEVICE Item item_at(const PrefillParams &p, const int *perm, int idx) {
   Item it;
-  if (p.group % 2 == 0) {
-    const int hp_n = p.h_q / 2, per = p.batch * hp_n;
-    const int rr = idx / per, rem = idx - rr * per;
-    it.b = rem / hp_n;
-    const int hp = rem - it.b * hp_n;
+  const bool even = p.group % 2 == 0;
+  const int n_in = even ? p.h_q / 2 : p.h_q;                   // items per (sequence, block step)
+  const int n_rr = even ? p.qb_max : (p.qb_max + 1) / 2;       // block steps per sequence
+  int bs, rr, h;
+  if (p.seq_major) {
+    const int per = n_rr * n_in;
+    bs = idx / per;
+    const int rem = idx - bs * per;
+    rr = rem / n_in;
+    h = rem - rr * n_in;
+  } else {
+    const int per = p.batch * n_in;
+    rr = idx / per;
+    const int rem = idx - rr * per;
+    bs = rem / n_in;
+    h = rem - bs * n_in;
+  }
+  it.b = ranked(p) ? perm[bs] : bs;
+  if (even) {
     const int r = p.qb_max - 1 - rr;
-    it.hq[0] = 2 * hp;
-    it.hq[1] = 2 * hp + 1;
+    it.hq[0] = 2 * h;
+    it.hq[1] = 2 * h + 1;
     it.r[0] = r;
     it.r[1] = r;
   } else {
-    const int qbp = (p.qb_max + 1) / 2, per = p.batch * p.h_q;
-    const int rr = idx / per, rem = idx - rr * per;
-    it.b = rem / p.h_q;
-    const int h = rem - it.b * p.h_q;
-    const int rp = qbp - 1 - rr;
+    const int rp = n_rr - 1 - rr;
     it.hq[0] = h;
     it.hq[1] = h;
     it.r[0] = 2 * rp;
@@ -328,6 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // after that read.
   volatile uint32_t *votes = misc + 4;          // [kNQ][3][4]
   volatile int *ring = reinterpret_cast<volatile int *>(misc + 28);   // [kSchedDepth] claimed items
+  // ranked sequences (written once, before the first claimed item is
+  // published; a static array, so that its address takes no register)
+  __shared__ int perm[kRankMax];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = num_items(p);
@@ -400,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t n = 0; ok; ++n) {
         const int idx = pop_warp(n);
         if (idx < 0) break;
-        const Item it = item_at(p, idx);
+        const Item it = item_at(p, perm, idx);
         const Seq sq = seq_at(p, it.b);
         if (sq.bad) continue;
         TileGeo g[kNQ];
@@ -425,8 +451,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int hk = it.hq[0] / p.group;
         const int32_t *bt = p.paged ? p.block_table + (size_t)it.b * p.max_pages : nullptr;
+        // a paged tile's block-table entries are read one tile ahead, so that
+        // their latency is not added to the copies' once the stage frees up
+        auto page_raw = [&](int j) -> int {
+          const int tok = j * BN + lane * kPageSize;
+          return (p.paged && lane < BN / kPageSize && tok < sq.s_k) ? __ldg(bt + tok / kPageSize) : 0;
+        };
+        int raw_next = page_raw(0);
         for (int j = 0; j < nmax; ++j, ++kv_c) {
           const int s = kv_c % kStages;
+          const int raw = raw_next;
+          if (j + 1 < nmax) raw_next = page_raw(j + 1);
           if (kv_c >= kStages && !(ok = wait_all_p(&kv_empty[s], ((kv_c / kStages) - 1) & 1))) break;
           if (lane == 0) {
             mbar_arrive_expect_tx(&k_full[s], BN * D * 2);
@@ -449,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int tok = j * BN + lane * kPageSize;
             int page = p.num_pages;
             if (tok < sq.s_k) {
-              page = __ldg(bt + tok / kPageSize);
+              page = raw;
               if (page < 0 || page >= p.num_pages) {
                 raise_error(p.err, ATTN_DEVERR_BLOCK_TABLE);
                 page = p.num_pages;
@@ -521,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (uint32_t n = 0; ok; ++n) {
       const int idx = pop_warp(n);
       if (idx < 0) break;
-      const Item it = item_at(p, idx);
+      const Item it = item_at(p, perm, idx);
       const Seq sq = seq_at(p, it.b);
       if (sq.bad) continue;
       TileGeo g[kNQ];
@@ -628,13 +663,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tile_c[t] > 0) drain(&o_done[t], (tile_c[t] - 1) & 1);
   } else if (warp == kSchedWarp) {
     // =============== work claims ===============
+    if (ranked(p)) {
+      // rank the sequences by key length, longest first, ties in index
+      // order, broken ones last; lane b holds sequence b, lane 0 writes the
+      // ranking
+      int key = INT_MIN;
+      if (lane < p.batch) {
+        const Seq sq = seq_at(p, lane);
+        key = sq.bad ? INT_MIN + 1 : sq.s_k;
+      }
+      int rank = 0;
+      for (int j = 0; j < p.batch; ++j) {
+        const int kj = __shfl_sync(0xffffffffu, key, j);
+        rank += (kj > key) || (kj == key && j < lane);
+      }
+      for (int r = 0; r < p.batch; ++r) {
+        const unsigned int m = __ballot_sync(0xffffffffu, lane < p.batch && rank == r);
+        if (lane == 0) perm[r] = __ffs(m) - 1;
+      }
+    }
     if (lane == 0) {
       unsigned int *next_item = &g_work[p.work_slot][0];
       // an item holds work when one of its query tiles holds rows (a tile
       // whose rows see no key still writes zeros and -inf); items of a
       // sequence with broken cu_seqlens are reported and dropped here
       auto has_work = [&](int idx) {
-        const Item it = item_at(p, idx);
+        const Item it = item_at(p, perm, idx);
         const Seq sq = seq_at(p, it.b);
         if (sq.bad) {
           raise_error(p.err, ATTN_DEVERR_CU_SEQLENS);
@@ -677,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (uint32_t n = 0; alive; ++n) {
       const int idx = pop_warp(n);
       if (idx < 0) break;
-      const Item it = item_at(p, idx);
+      const Item it = item_at(p, perm, idx);
       const Seq sq = seq_at(p, it.b);
       const TileGeo g = tile_geo(p, sq, it.r[t]);
       if (!g.active) continue;

@@ -135,3 +135,19 @@ def test_bad_block_table_entry(A):
     _run(A, data, True, t=t)
     err = A.attn_get_last_device_error()
     assert err & 4, err                      # ATTN_DEVERR_BLOCK_TABLE
+
+
+@pytest.mark.parametrize("n_seq", [31, 32, 33, 45])
+def test_many_sequences(A, n_seq):
+    """Work items are ranked by sequence length for batches of up to 32
+    sequences and taken in batch order beyond; both sides of that limit, with
+    contexts longer than the queries (sequences outermost in the item order)
+    and a few empty queries or contexts."""
+    rng = np.random.default_rng(40 + n_seq)
+    lens_q = rng.integers(0, 150, n_seq)
+    lens_k = lens_q + rng.integers(0, 400, n_seq)
+    lens_k[3] = 0
+    lens_q[3] = 0
+    lens_q[5] = 0
+    data = W.paged_prefill(lens_q.tolist(), lens_k.tolist(), h_q=4, h_kv=2, d=64, seed=50 + n_seq)
+    _check(A, data, True)
