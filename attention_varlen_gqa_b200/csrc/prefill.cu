@@ -315,6 +315,28 @@ ATTN_DEVICE void exp64_to_tmem(const uint32_t (&a)[32], const uint32_t (&b)[32],
   ps[1] = x0 + x1;
 }
 
+// p = 2^(s * sl2 - mref) for one 32-column sub-tile of a row, packed to bf16
+// pairs and stored to TMEM at `taddr` (16 columns); returns the sum of p
+// (the same pairing as exp64_to_tmem's per-chunk sums).
+ATTN_DEVICE float exp32_to_tmem(const uint32_t (&a)[32], float sl2, float mref, uint32_t taddr) {
+  const uint64_t scale2 = f2_pack(sl2, sl2), neg_m2 = f2_pack(-mref, -mref);
+  uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+  uint32_t pk[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1])), scale2, neg_m2);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    acc[q & 1] = f2_add(acc[q & 1], f2_pack(p0, p1));
+    pk[q] = pack_bf16x2(p0, p1);
+  }
+  tmem_st16(taddr, pk);
+  float x0, x1;
+  f2_unpack(f2_add(acc[0], acc[1]), x0, x1);
+  return x0 + x1;
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -345,10 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
   // skip votes of the four warps of a softmax warpgroup, per query tile and
   // tile count mod 3: bit u = every row of the warp votes to skip 32-key
-  // sub-tile u.  Three slots: a warp may reach tile c + 1 while a slower warp
-  // of its group still reads the votes of tile c - 1, but no warp writes tile
-  // c + 2's before every warp has handed over P of tile c + 1, which comes
-  // after that read.
+  // sub-tile u.  The warps read tile c's votes right after its votes_ready
+  // phase and the MMA warp before it issues tile c's P.V; tile c + 3's votes
+  // (the same slot) come after S of tile c + 3, which follows all of those.
   volatile uint32_t *votes = misc + 4;          // [kNQ][3][4]
   volatile int *ring = reinterpret_cast<volatile int *>(misc + 28);   // [kSchedDepth] claimed items
   // ranked sequences (written once, before the first claimed item is
@@ -587,9 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Skip-softmax: the four softmax warps' votes for this tile were
           // written before their P hand-off; a 32-key sub-tile is skipped when
           // every row votes for it, and its P.V MMAs (two 16-key steps) are not
-          // issued.  The softmax warps take the skipped keys' p out of their
-          // row sums one tile later.
-          // (sub-tiles past the keys vote skip too: their p is 0 either way)
+          // issued (the softmax warps wrote no P for it and left it out of
+          // their row sums; sub-tiles past the keys vote skip too).
           uint32_t skip_bits = 0;
           if constexpr (SKIP) skip_bits = and4_shared(votes + (t * 3 + vslot[t]) * 4);
           if (!v_ready) {
@@ -745,45 +765,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       bool pv_any = false;
 
-      // One K/V tile: the four 32-key sub-tile maxima, the
-      // running max and lazy rescale (and the skip votes), then the
-      // exponentials in two halves; P of keys [0, 64) is handed to the MMA
-      // warp before the second half is computed, so the first half of P.V
-      // overlaps it.  (Starting the first half's exponentials before the
-      // maxima, with a redo when a row's max grew, measured 6 % slower: the
-      // maxima then trailed the exponentials on the path to the hand-off.)
-      // p summed per 32-key sub-tile over the row's last tile, and the
-      // correction once that tile's skip decisions are known: the skipped
-      // keys' p leave the row sum (their P.V MMAs were never issued)
-      float ps[4] = {0.f, 0.f, 0.f, 0.f}, ps_prev[4] = {0.f, 0.f, 0.f, 0.f};
-      // drop the skipped keys of the tile with warpgroup count c, local index
-      // jp, whose sub-tile sums are q, now worth `scale` each; the first warp
-      // also counts and records the skipped units
-      auto drop_skipped = [&](uint32_t c, int jp, const float (&q)[4], float scale) {
-        alive = alive && __all_sync(0xffffffffu, wait_or_abort(&votes_ready[2 * t + (c & 1)], (c >> 1) & 1,
-                                                               abort_flag, p.err));
-        uint32_t skip = and4_shared(votes + (t * 3 + c % 3) * 4);
-        float d = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool vis = jp * BN + 32 * u < g.k_end;
-          if (((skip >> u) & 1u) && vis) d += q[u];
-          if (!vis) skip &= ~(1u << u);
-        }
-        l -= d * scale;
-        if (quad == 0 && skip != 0) {
-          n_skip += __popc(skip);
-          if (lane == 0 && p.skip_mask) {
-            for (int u = 0; u < 4; ++u) {
-              if ((skip >> u) & 1u) {
-                const long long unit = (((long long)it.b * p.qb_max + it.r[t]) * p.h_q + hq) * p.kt_max +
-                                       (jp * BN / 32 + u);
-                atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
-              }
-            }
-          }
-        }
-      };
+      // One K/V tile: the four 32-key sub-tile maxima, the running max and
+      // lazy rescale, then the exponentials in two halves; P of keys [0, 64)
+      // is handed to the MMA warp before the second half is computed, so the
+      // first half of P.V overlaps it.  (Starting the first half's
+      // exponentials before the maxima, with a redo when a row's max grew,
+      // measured 6 % slower: the maxima then trailed the exponentials on the
+      // path to the hand-off.)  Skip mode: each warp votes per 32-key
+      // sub-tile from its rows' maxima; the four votes are combined before
+      // the exponentials, and a skipped sub-tile gets none: its p are 0, it
+      // adds nothing to the row sums, and the MMA warp issues no P.V for it.
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       if (SKIP && quad == 0 && g.n > 0) n_vis += (g.k_end + kSkipTile - 1) / kSkipTile;
       auto step = [&](int j) -> bool {
         const bool ok =
@@ -804,10 +796,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mref = (m_used == -INFINITY) ? 0.f : m_used;
         float um[4];                                // raw maxima of the four 32-key sub-tiles
         max_sub4(sr, um);
-        uint32_t wv = 0;                            // the warp's skip votes (bit u: sub-tile u)
         if constexpr (SKIP) {
           // vote per 32-key sub-tile: exp(sub-tile max - running max) <
-          // threshold; the MMA warp combines the four warps' votes
+          // threshold for every row of the warp
           uint32_t my_votes = 0;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -816,10 +807,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_true = fmaxf(m_true, t2);
             my_votes |= uint32_t(vote) << u;
           }
-          // stored with the P hand-off below (which orders it for the MMA
-          // warp; the warpgroup's own readers wait on votes_ready), so the
-          // reduction overlaps the exponentials
-          wv = __reduce_and_sync(0xffffffffu, my_votes);
+          const uint32_t wv = __reduce_and_sync(0xffffffffu, my_votes);
+          if (lane == 0) {
+            votes[(t * 3 + tile_c % 3) * 4 + quad] = wv;
+            mbar_arrive(&votes_ready[2 * t + (tile_c & 1)]);
+          }
         } else {
           m_true = fmaxf(m_true, fmaxf(fmaxf(um[0], um[1]), fmaxf(um[2], um[3])) * sl2);
         }
@@ -831,7 +823,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_true;
           mref = m_used;
         }
-        exp64_to_tmem(sr[0], sr[1], sl2, mref, tS, ps);
+        uint32_t skip = 0;                          // sub-tiles every row of the warpgroup skips
+        if constexpr (SKIP) {
+          // the four warps' votes (a warp is at most one tile ahead of the
+          // others: the next S needs every warp's P of this one)
+          if (!__all_sync(0xffffffffu, wait_or_abort(&votes_ready[2 * t + (tile_c & 1)], (tile_c >> 1) & 1,
+                                                     abort_flag, p.err))) {
+            alive = false;
+            return false;
+          }
+          skip = and4_shared(votes + (t * 3 + tile_c % 3) * 4);
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            ps[u] = ((skip >> u) & 1u) ? 0.f : exp32_to_tmem(sr[u], sl2, mref, tS + 16 * u);
+        } else {
+          exp64_to_tmem(sr[0], sr[1], sl2, mref, tS, ps);
+        }
         // rescale the O accumulator rows whose reference max moved
         if (pv_any && __any_sync(0xffffffffu, alpha != 1.f)) {
           const bool okw =
@@ -854,25 +861,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          if (SKIP) votes[(t * 3 + tile_c % 3) * 4 + quad] = wv;
-          mbar_arrive(&p_half[t]);
-          if (SKIP) mbar_arrive(&votes_ready[2 * t + (tile_c & 1)]);
+        if (lane == 0) mbar_arrive(&p_half[t]);
+        if constexpr (SKIP) {
+#pragma unroll
+          for (int u = 2; u < 4; ++u)
+            ps[u] = ((skip >> u) & 1u) ? 0.f : exp32_to_tmem(sr[u], sl2, mref, tS + 16 * u);
+        } else {
+          exp64_to_tmem(sr[2], sr[3], sl2, mref, tS + 32, ps + 2);
         }
-        exp64_to_tmem(sr[2], sr[3], sl2, mref, tS + 32, ps + 2);
         l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[t]);
+        if constexpr (SKIP) {
+          // count and record the skipped units (sub-tiles past the keys vote
+          // skip too, but are not units)
+          if (quad == 0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (j * BN + 32 * u >= g.k_end) skip &= ~(1u << u);
+            n_skip += __popc(skip);
+            if (lane == 0 && p.skip_mask && skip != 0) {
+              for (int u = 0; u < 4; ++u) {
+                if ((skip >> u) & 1u) {
+                  const long long unit = (((long long)it.b * p.qb_max + it.r[t]) * p.h_q + hq) * p.kt_max +
+                                         (j * BN / 32 + u);
+                  atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
+                }
+              }
+            }
+          }
+        }
         ++tile_c;
         pv_any = true;
-        if constexpr (SKIP) {
-          // the previous tile's decisions are known by now
-          if (j > 0) drop_skipped(tile_c - 2, j - 1, ps_prev, alpha);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) ps_prev[u] = ps[u];
-        }
         return alive;
       };
 
@@ -881,8 +903,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!alive) break;
 
       // ---------------- epilogue ----------------
-      if (SKIP && g.n > 0) drop_skipped(tile_c - 1, g.n - 1, ps_prev, 1.f);
-      if (!alive) break;
       const bool have_o = g.n > 0;
       if (have_o) {
         alive = __all_sync(0xffffffffu, wait_or_abort(&o_done[t], (tile_c - 1) & 1, abort_flag, p.err));

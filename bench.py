@@ -15,7 +15,10 @@ The headline `value` is the prefill throughput (TFLOP/s over the allowed
 operation's inputs are larger than the 126 MB L2, so no flush is needed
 between steps.  The skip-softmax workload (4 x 16384 prefill, batch 32 x
 32768 decode, peaked sink/window keys) is measured after the timed steps at
-thresholds {0, 1e-3, 1e-2, 0.1} and reported with its skipped-unit fraction.
+thresholds {0, 1e-3, 1e-2, 0.1} and reported with its skipped-unit fraction;
+so is an attention-sink workload on the same shapes (strong sink keys that
+most query rows align with), on which most tiles are skipped, to show what
+skipping saves.
 
 Multi-GPU (torchrun, one rank per GPU): the operations are independent
 problems, so every rank runs the same step on its own seed (weak scaling, no
@@ -52,7 +55,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip", "smallseq_bwd",
-                                       "decode_skip", "varlen_bwd"],
+                                       "decode_skip", "varlen_bwd", "paged_prefill"],
                     default="all",
                     help="profiling aid: run a single operation (no JSON line)")
     ap.add_argument("--no-skip", action="store_true",
@@ -350,6 +353,10 @@ def main():
     if args.only == "skip":
         measure_skip(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
         return
+    if args.only == "paged_prefill":
+        measure_paged_prefill(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
+        assert A.attn_get_last_device_error() == 0
+        return
     if args.only == "varlen_bwd":
         measure_varlen_bwd(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
         assert A.attn_get_last_device_error() == 0
@@ -500,74 +507,97 @@ def main():
         dist.destroy_process_group()
 
 
-def measure_skip(A, W, torch, dev, seed, pk, reps=3):
-    """Skip-softmax workload at thresholds {0, 1e-3, 1e-2, 0.1}."""
-    import numpy as np
-    res = {"prefill": {}, "decode": {}}
-    sp = W.skip_prefill(seed=seed, where="device")
+def _time_ms(torch, run, reps):
+    run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def _skip_prefill_sweep(A, torch, dev, sp, reps, thresholds):
     cq = torch.from_numpy(sp["cu_seqlens_q"]).to(dev)
     ck = torch.from_numpy(sp["cu_seqlens_k"]).to(dev)
     out = torch.empty_like(sp["q"])
     lse = torch.empty(sp["q"].shape[:2], dtype=torch.float32, device=dev)
     counts = torch.zeros(2, dtype=torch.int64, device=dev)
-    dense_flops = prefill_flops(sp["lens_q"], sp["lens_k"], 32, 128, True)
-    for thr in (0.0, 1e-3, 1e-2, 0.1):
+    dense_flops = prefill_flops(sp["lens_q"], sp["lens_k"], sp["h_q"], sp["d"], True)
+    res = {}
+    for thr in thresholds:
         def run():
             A.attn_varlen_fwd(sp["q"], sp["k"], sp["v"], cq, ck, sp["max_q"], sp["max_k"], causal=True,
                               out=out, lse=lse, skip_threshold=thr, skip_counts=counts)
-        run()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            run()
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / reps
+        ms = _time_ms(torch, run, reps)
         vis, sk = (int(x) for x in counts.tolist())
         frac = sk / vis if vis and thr > 0 else 0.0
         # executed: QK^T over visited units always, PV only over kept ones
         executed = dense_flops * (1.0 - frac / 2.0)
-        res["prefill"][str(thr)] = {"ms": ms, "skipped_frac": frac, "visited_units": vis,
-                                    "skipped_units": sk,
-                                    "dense_equiv_tflops": dense_flops / ms / 1e9,
-                                    "executed_tflops_est": executed / ms / 1e9}
-    del sp, out, lse
-    sd = W.skip_decode(seed=seed, where="device")
+        res[str(thr)] = {"ms": ms, "skipped_frac": frac, "visited_units": vis, "skipped_units": sk,
+                         "dense_equiv_tflops": dense_flops / ms / 1e9, "executed_tflops_est": executed / ms / 1e9}
+    return res
+
+
+def _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs):
+    """runs: (key, threshold, schedule) triples."""
+    import numpy as np
     bt = torch.from_numpy(sd["block_table"]).to(dev)
     sl = torch.from_numpy(sd["seq_lens"]).to(dev)
-    dout = torch.empty_like(sd["q"])
-    dlse = torch.empty(sd["q"].shape[:2], dtype=torch.float32, device=dev)
-    Ls = sd["seq_lens"].astype(np.int64)
-    kbytes = float(Ls.sum() * 8 * 128 * 2)
-    # skip mode: the two-pass schedule (workspace given); "0.1/sequential" is the
-    # one-split-per-(sequence, kv-head) schedule at the same threshold
-    for key, thr, sched in ((0.0, 0.0, "split"), (1e-3, 1e-3, "split"), (1e-2, 1e-2, "split"),
-                            (0.1, 0.1, "split"), ("0.1/sequential", 0.1, "sequential")):
+    B, h_q, d = sd["q"].shape
+    h_kv = sd["k_cache"].shape[2]
+    out = torch.empty_like(sd["q"])
+    lse = torch.empty((B, h_q), dtype=torch.float32, device=dev)
+    counts = torch.zeros(2, dtype=torch.int64, device=dev)
+    kbytes = float(sd["seq_lens"].astype(np.int64).sum() * h_kv * d * 2)
+    res = {}
+    for key, thr, sched in runs:
         ws = None
         if sched == "split":
-            ws = torch.empty(A.attn_paged_decode_workspace_size(32, 32, 128, bt.shape[1], thr), dtype=torch.uint8,
+            ws = torch.empty(A.attn_paged_decode_workspace_size(B, h_q, d, bt.shape[1], thr), dtype=torch.uint8,
                              device=dev)
 
         def run():
             A.attn_paged_decode(sd["q"], sd["k_cache"], sd["v_cache"], bt, sl, skip_threshold=thr,
-                                out=dout, lse=dlse, workspace=ws, skip_counts=counts, skip_schedule=sched)
-        run()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            run()
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / reps
+                                out=out, lse=lse, workspace=ws, skip_counts=counts, skip_schedule=sched)
+        ms = _time_ms(torch, run, reps)
         vis, sk = (int(x) for x in counts.tolist())
         frac = sk / vis if vis and thr > 0 else 0.0
-        alg = kbytes + kbytes * (1.0 - frac) + 32 * 32 * 128 * 2 * 2 + 32 * 32 * 4
-        res["decode"][str(key)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
-                                   "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"],
-                                   "schedule": "dense split-KV" if thr == 0 else
-                                   ("two passes over 32 splits" if sched == "split" else "one sequential split")}
+        # all of K, V of the kept tiles, q, out and lse
+        alg = kbytes + kbytes * (1.0 - frac) + B * h_q * d * 2 * 2 + B * h_q * 4
+        res[str(key)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
+                         "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"],
+                         "schedule": "dense split-KV" if thr == 0 else
+                         ("two passes over 32 splits" if sched == "split" else "one sequential split")}
+    return res
+
+
+def measure_skip(A, W, torch, dev, seed, pk, reps=3):
+    """Skip-softmax workload at thresholds {0, 1e-3, 1e-2, 0.1}, plus the
+    attention-sink workload on the same shapes, on which most tiles pass the
+    skip test (what skipping saves)."""
+    thresholds = (0.0, 1e-3, 1e-2, 0.1)
+    # skip mode runs the two-pass schedule (workspace given); "0.1/sequential"
+    # is the one-split-per-(sequence, kv-head) schedule at the same threshold
+    runs = [(t, t, "split") for t in thresholds] + [("0.1/sequential", 0.1, "sequential")]
+    res = {}
+    sp = W.skip_prefill(seed=seed, where="device")
+    res["prefill"] = _skip_prefill_sweep(A, torch, dev, sp, reps, thresholds)
+    del sp
+    sd = W.skip_decode(seed=seed, where="device")
+    res["decode"] = _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs)
+    del sd
+    sink = {"workload": "attention sinks (not a pages workload): the same shapes; per kv-head a unit "
+                        "direction u, q += sqrt(d) u, the first 4 keys of each sequence k += 12 u"}
+    sp = W.sink_prefill(seed=seed, where="device")
+    sink["prefill"] = _skip_prefill_sweep(A, torch, dev, sp, reps, thresholds)
+    del sp
+    sd = W.sink_decode(seed=seed, where="device")
+    sink["decode"] = _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs)
+    del sd
+    res["sink"] = sink
     return res
 
 

@@ -236,3 +236,15 @@ def test_full_size_skip_sampled(A, thr, schedule):
     data = W.skip_decode(seed=0, where="device")
     batches = [0, 13, 31]
     _check(A, data, thr, t=_dev(data), batches=batches, host=_sampled_host(data, batches), schedule=schedule)
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+@pytest.mark.parametrize("thr", [1e-3, 1e-2])
+def test_full_size_sink_sampled(A, thr, schedule):
+    """Batch 32 at 32768 keys with strong attention sinks, where nearly every
+    tile is skipped; 2 sampled sequences vs the oracle, skip sets included."""
+    data = W.sink_decode(seed=0, where="device")
+    batches = [3, 30]
+    vis, skipped = _check(A, data, thr, t=_dev(data), batches=batches, host=_sampled_host(data, batches),
+                          schedule=schedule)
+    assert skipped > vis // 2

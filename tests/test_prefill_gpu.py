@@ -209,6 +209,15 @@ def test_full_size_skip_prefill_sampled(A, thr):
     assert int(counts[0]) > 0
 
 
+@pytest.mark.parametrize("thr", [1e-3, 1e-2])
+def test_full_size_sink_prefill_sampled(A, thr):
+    """4 x 16384 causal with strong attention sinks, where most units are
+    skipped; sequence 1, kv-head 5."""
+    data = W.sink_prefill(seed=0, where="device")
+    counts = _check_sampled(A, data, thr, [1], 5)
+    assert int(counts[1]) > int(counts[0]) // 4
+
+
 def test_concurrent_calls_and_counter_reuse(A):
     """The kernel's CTAs claim work from a per-call counter (64 per device,
     taken in turn and re-zeroed by the kernel).  Two calls in flight on two

@@ -278,6 +278,65 @@ def skip_parity_prefill(lens, h_q=4, h_kv=2, d=64, seed=0, spread=0.25, peak=6.0
                 scale=1.0 / np.sqrt(d), values="host", seed=seed)
 
 
+def _sink_directions(seed, h_kv, d):
+    rng = np.random.default_rng(seed + 7919)
+    u = rng.standard_normal((h_kv, d))
+    return (u / np.linalg.norm(u, axis=1, keepdims=True)).astype(np.float32)
+
+
+def _add_rows(x, rows, heads, delta, where):
+    """x[rows, heads] += delta (bf16 buffer: host uint16 bits or a device tensor)."""
+    if where == "host":
+        xf = bf16_bits_to_f32(x)
+        xf[np.ix_(rows, heads)] += delta
+        return f32_to_bf16_bits(xf)
+    import torch
+    r = torch.as_tensor(rows, device=x.device).view(-1, 1)
+    h = torch.as_tensor(heads, device=x.device).view(1, -1)
+    x[r, h] = (x[r, h].float() + torch.as_tensor(delta, device=x.device)).to(x.dtype)
+    return x
+
+
+def sink_prefill(seed=0, n_seq=4, L=16384, h_q=32, h_kv=8, d=128, n_sink=4, beta=12.0, where="device"):
+    """Attention-sink prefill, a workload of this package (not one the pages
+    measure) on which the skip rule has work to skip: per kv-head a seeded
+    unit direction u; every query row is N(0, 1) + sqrt(d) u of its kv-head
+    and the first ``n_sink`` keys of each sequence get k += beta u, so their
+    scaled scores sit near beta while all other scores are about N(0, 2)."""
+    data = varlen_prefill([L] * n_seq, h_q=h_q, h_kv=h_kv, d=d, causal=True, seed=seed, where=where)
+    u = _sink_directions(seed, h_kv, d)
+    G = h_q // h_kv
+    rows_q = np.arange(int(data["cu_seqlens_q"][-1]))
+    data["q"] = _add_rows(data["q"], rows_q, np.arange(h_q), np.repeat(u, G, axis=0)[None] * np.sqrt(d), where)
+    sinks = np.concatenate([int(c) + np.arange(n_sink) for c in data["cu_seqlens_k"][:-1]])
+    data["k"] = _add_rows(data["k"], sinks, np.arange(h_kv), (beta * u)[None], where)
+    data["peaks"] = dict(n_sink=n_sink, beta=beta)
+    return data
+
+
+def sink_decode(seed=0, batch=32, L=32768, h_q=32, h_kv=8, d=128, page_size=16, n_sink=4, beta=12.0,
+                where="device"):
+    """The attention-sink recipe of ``sink_prefill`` on the paged decode
+    shapes: q += sqrt(d) u of its kv-head, the first ``n_sink`` cache
+    positions of every sequence get k += beta u."""
+    data = paged_decode([L] * batch, h_q=h_q, h_kv=h_kv, d=d, page_size=page_size, seed=seed, where=where)
+    u = _sink_directions(seed, h_kv, d)
+    G = h_q // h_kv
+    B = len(data["seq_lens"])
+    q2 = data["q"].reshape(B, h_q, d) if where == "host" else data["q"]
+    data["q"] = _add_rows(q2, np.arange(B), np.arange(h_q), np.repeat(u, G, axis=0)[None] * np.sqrt(d), where)
+    kc = data["k_cache"]
+    shape = kc.shape
+    flat = kc.reshape(shape[0] * shape[1], h_kv, d)
+    pos = np.arange(n_sink)
+    slots = np.concatenate([data["block_table"][b, pos // page_size].astype(np.int64) * page_size
+                            + pos % page_size for b in range(B)])
+    flat = _add_rows(flat, slots, np.arange(h_kv), (beta * u)[None], where)
+    data["k_cache"] = flat.reshape(shape)
+    data["peaks"] = dict(n_sink=n_sink, beta=beta)
+    return data
+
+
 # ---------------------------------------------------------------------------
 # Small-seq cross attention
 # ---------------------------------------------------------------------------
