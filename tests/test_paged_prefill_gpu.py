@@ -151,3 +151,28 @@ def test_many_sequences(A, n_seq):
     lens_q[5] = 0
     data = W.paged_prefill(lens_q.tolist(), lens_k.tolist(), h_q=4, h_kv=2, d=64, seed=50 + n_seq)
     _check(A, data, True)
+
+
+def test_bad_seq_len_in_ranked_batch(A):
+    """Sequences outermost and ranked (keys beyond queries, 5 sequences): one
+    seq_lens_k entry beyond its block-table row is reported and its rows are
+    left alone; the other sequences are exact."""
+    data = W.paged_prefill([30, 64, 5, 100, 17], [200, 64, 300, 400, 17], h_q=4, h_kv=2, d=64, seed=37)
+    t = _dev(data)
+    bad = 2
+    t["sl"][bad] = data["block_table"].shape[1] * 16 + 1
+    out0 = torch.full_like(t["q"], 3.0)
+    out, lse = A.attn_paged_prefill(t["q"], t["k_cache"], t["v_cache"], t["bt"], t["cu_q"], t["sl"],
+                                    data["max_q"], data["block_table"].shape[1] * 16 + 1, causal=True,
+                                    scale=data["scale"], out=out0)
+    err = A.attn_get_last_device_error()
+    assert err & 1, err                      # ATTN_DEVERR_CU_SEQLENS
+    ro, rl, _ = oracle.paged_prefill(data["q"], data["k_cache"], data["v_cache"], data["block_table"],
+                                     data["cu_seqlens_q"], data["seq_lens_k"], data["h_q"], data["h_kv"], True,
+                                     data["scale"])
+    cu = data["cu_seqlens_q"]
+    good = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in range(5) if b != bad])
+    gsel = torch.as_tensor(good, device="cuda")
+    assert_close_bf16(out[gsel], ro[good])
+    assert_close_lse(lse[gsel], rl[good])
+    assert torch.all(out[int(cu[bad]):int(cu[bad + 1])] == 3.0)
