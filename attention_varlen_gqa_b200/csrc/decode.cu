@@ -596,7 +596,8 @@ struct PassLayout {
   // pass 1: [2][warp][16] 16-key maxima; pass 2: [split][G] the earlier splits' maxima
   static constexpr int kX = kStages * kStage;
   static constexpr int kTmax = kX + kDecodeSplits * kMaxGroup * 4;   // pass 2: the split's tile maxima
-  static constexpr int kKeep = kTmax + (PV ? kTmaxCap * 4 : 0);  // pass 2: [stage] decision bits
+  // pass 2: per stage the chunk's decision bits, then per stage its chunk index
+  static constexpr int kKeep = kTmax + (PV ? kTmaxCap * 4 : 0);
   static constexpr int kBar = kKeep + 8 * kStages;
   static constexpr int kBt = kBar + kStages * 8;
   static constexpr int kBtCap = 256;
@@ -824,8 +825,8 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
       }
       return kb;
     };
-    auto issue = [&](int c, uint32_t kb) {   // lane 0 of warp 0
-      const int s = c % Lay::kStages;
+    auto issue = [&](int i, int c, uint32_t kb) {   // lane 0 of warp 0: ring position i, chunk c
+      const int s = i % Lay::kStages;
       uint8_t *stage = base + s * Lay::kStage;
       const int tok0 = (r.c0 + c) * kChunk;
       const int npg = (min(r.L - tok0, kChunk) + kPageSize - 1) / kPageSize;
@@ -834,23 +835,56 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
       const int hi = min(npg, (kb & 2u) ? 4 : ((kb & 1u) ? 2 : 0));
       const uint32_t sbytes = kb ? kChunk * G * 4 : 0u;
       keep_s[s] = kb;
+      keep_s[Lay::kStages + s] = (uint32_t)c;
       mbar_arrive_expect_tx(&full[s], max(0, hi - lo) * (D / 64) * (16 * 64 * 2) + sbytes);
       issue_pages<D>(&vmap, stage, &full[s], r.pages, tok0, r.L, hk, lo, hi, false);
       if (sbytes) bulk_load(stage + Lay::kSlot, S + (size_t)tok0 * G, sbytes, &full[s]);
     };
-    int issued = 0;
-    if (ln.w == 0)
-      for (; issued < min(n, Lay::kStages); ++issued) {
-        const uint32_t kb = decide(issued);
-        if (ln.lane == 0) issue(issued, kb);
+    // Warp 0 decides the chunks in tile order and puts only the kept ones in
+    // the ring, each marked when no kept chunk follows (it decides one kept
+    // chunk ahead): a skipped chunk costs its decision, taken while the other
+    // warps work on earlier chunks, not a round of the ring.  A split with
+    // no kept chunk gets one end entry.
+    constexpr uint32_t kLast = 4u, kEndEntry = 0xffffffffu;
+    int next_c = 0;              // warp 0: the next chunk to decide
+    int pend_c = 0;              // warp 0: the next kept chunk and its tile bits (0: none)
+    uint32_t pend_kb = 0;
+    bool more = true;            // warp 0: the last entry is not issued yet
+    auto find_kept = [&]() {
+      pend_kb = 0;
+      while (pend_kb == 0 && next_c < n) {
+        pend_c = next_c++;
+        pend_kb = decide(pend_c);
       }
-    for (int i = 0; i < n; ++i) {
+    };
+    auto next_issue = [&](int i) {   // warp 0: ring position i
+      const int c = pend_c;
+      const uint32_t kb = pend_kb;
+      if (kb) find_kept();
+      if (ln.lane == 0) {
+        if (kb) {
+          issue(i, c, kb | (pend_kb ? 0u : kLast));
+        } else {
+          keep_s[i % Lay::kStages] = kEndEntry;
+          mbar_arrive(&full[i % Lay::kStages]);
+        }
+      }
+      more = kb != 0 && pend_kb != 0;
+    };
+    int issued = 0;
+    if (ln.w == 0) {
+      find_kept();
+      for (; more && issued < Lay::kStages; ++issued) next_issue(issued);
+    }
+    for (int i = 0;; ++i) {
       const int s = i % Lay::kStages;
       const bool ok = mbar_wait(&full[s], (i / Lay::kStages) & 1, p.err);
+      bool ended = false;
       if (ok) {
         const uint32_t kb = keep_s[s];
-        const int tok_base = (r.c0 + i) * kChunk + ln.w * 16;
-        if (((kb >> (ln.w >> 1)) & 1u) && tok_base < r.L) {
+        ended = kb == kEndEntry || (kb & kLast);
+        const int tok_base = (r.c0 + (int)keep_s[Lay::kStages + s]) * kChunk + ln.w * 16;
+        if (kb != kEndEntry && ((kb >> (ln.w >> 1)) & 1u) && tok_base < r.L) {
           const uint32_t vslot = sbase + s * Lay::kStage;
           const float *ss = reinterpret_cast<const float *>(base + s * Lay::kStage + Lay::kSlot);
           float sc[NH][4], qm[NH][2];
@@ -879,10 +913,10 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
         failed = true;
         break;
       }
+      if (ended) break;
       // every warp is done with stage s
-      if (ln.w == 0 && issued < n) {
-        const uint32_t kb = decide(issued);
-        if (ln.lane == 0) issue(issued, kb);
+      if (ln.w == 0 && more) {
+        next_issue(issued);
         ++issued;
       }
     }
