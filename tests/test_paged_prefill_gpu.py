@@ -176,3 +176,25 @@ def test_bad_seq_len_in_ranked_batch(A):
     assert_close_bf16(out[gsel], ro[good])
     assert_close_lse(lse[gsel], rl[good])
     assert torch.all(out[int(cu[bad]):int(cu[bad + 1])] == 3.0)
+
+
+def test_sequence_order_does_not_change_results(A):
+    """The same sequences in reverse batch order (so the longest-first ranking
+    and the claim order both change): every sequence's output and LSE are
+    bit-identical to the forward order's."""
+    lens_q = [40, 130, 7, 256, 65, 1]
+    lens_k = [300, 130, 900, 700, 65, 1500]
+    data = W.paged_prefill(lens_q, lens_k, h_q=8, h_kv=2, d=128, seed=38)
+    t = _dev(data)
+    out, lse, *_ = _run(A, data, True, t=t)
+    order = list(range(len(lens_q)))[::-1]
+    cu = data["cu_seqlens_q"]
+    rows = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in order])
+    ridx = torch.as_tensor(rows, device="cuda")
+    cu_r = dev_i32(W.cu_from_lens([lens_q[b] for b in order]))
+    bt_r = t["bt"][torch.as_tensor(order, device="cuda")].contiguous()
+    sl_r = t["sl"][torch.as_tensor(order, device="cuda")].contiguous()
+    out_r, lse_r = A.attn_paged_prefill(t["q"][ridx].contiguous(), t["k_cache"], t["v_cache"], bt_r, cu_r, sl_r,
+                                        data["max_q"], data["max_k"], causal=True, scale=data["scale"])
+    assert A.attn_get_last_device_error() == 0
+    assert torch.equal(out_r, out[ridx]) and torch.equal(lse_r, lse[ridx])
