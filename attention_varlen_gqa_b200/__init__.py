@@ -52,7 +52,7 @@ for _name, (_res, _args) in EXPORTS.items():
     _fn.restype = _res
     _fn.argtypes = _args
 
-DEVERR = {1: "CU_SEQLENS", 2: "SEQ_LEN", 4: "BLOCK_TABLE", 8: "SMALLSEQ_LEN", 16: "TIMEOUT"}
+DEVERR = {1: "CU_SEQLENS", 2: "SEQ_LEN", 4: "BLOCK_TABLE", 8: "SMALLSEQ_LEN", 16: "TIMEOUT", 32: "BUSY"}
 
 
 class AttnError(RuntimeError):
@@ -132,10 +132,16 @@ def attn_varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_q, max_k, causal=Tr
     if lse is None and want_lse:
         lse = torch.empty((total_q, h_q), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib.attn_varlen_fwd_ex(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, total_q, total_k,
-        int(max_q), int(max_k), h_q, h_kv, d, int(bool(causal)), scale, float(skip_threshold),
-        _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _stream(stream))
+    if skip_threshold == 0.0 and skip_mask is None and skip_counts is None:
+        # the plain entry point when nothing of the skip-softmax extension is asked for
+        rc = lib.attn_varlen_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, total_q, total_k,
+            int(max_q), int(max_k), h_q, h_kv, d, int(bool(causal)), scale, _ptr(out), _ptr(lse), _stream(stream))
+    else:
+        rc = lib.attn_varlen_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, total_q, total_k,
+            int(max_q), int(max_k), h_q, h_kv, d, int(bool(causal)), scale, float(skip_threshold),
+            _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _stream(stream))
     _check("attn_varlen_fwd", rc)
     return out, lse
 
@@ -246,11 +252,18 @@ def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size=16, 
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         ws_bytes = workspace.numel() * workspace.element_size()
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib.attn_paged_decode_ex(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), batch, num_pages,
-        block_table.shape[1], page_size, h_q, h_kv, d, float(skip_threshold), scale,
-        _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
-        _stream(stream))
+    if skip_mask is None and skip_counts is None:
+        # the plain entry point when no skip reporting is asked for
+        rc = lib.attn_paged_decode(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), batch, num_pages,
+            block_table.shape[1], page_size, h_q, h_kv, d, float(skip_threshold), scale, _ptr(out), _ptr(lse),
+            _ptr(workspace), ws_bytes, _stream(stream))
+    else:
+        rc = lib.attn_paged_decode_ex(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), batch, num_pages,
+            block_table.shape[1], page_size, h_q, h_kv, d, float(skip_threshold), scale,
+            _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+            _stream(stream))
     _check("attn_paged_decode", rc)
     return out, lse
 

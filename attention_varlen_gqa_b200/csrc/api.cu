@@ -384,6 +384,25 @@ SkipWorkspace skip_workspace(int batch, int h_q, int d, int max_pages_per_seq) {
   return w;
 }
 
+// Host-checkable arguments of the paged decode entry points (everything but
+// the workspace), in the order their error codes are documented.
+int check_decode_args(const void *q, const void *k_cache, const void *v_cache, const void *block_table,
+                      const void *seq_lens, int batch, int num_pages, int max_pages_per_seq, int page_size,
+                      int h_q, int h_kv, int d, float skip_threshold, float scale, const void *out) {
+  if (batch < 0 || num_pages < 0 || max_pages_per_seq < 0) return ATTN_E_SHAPE;
+  if (page_size != kPageSize) return ATTN_E_PAGE_SIZE;
+  if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || h_q / h_kv > kMaxGroup) return ATTN_E_HEADS;
+  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
+  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
+  const int rc = check_threshold(skip_threshold);
+  if (rc) return rc;
+  if (batch > 0 && (num_pages <= 0 || max_pages_per_seq <= 0)) return ATTN_E_SHAPE;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return ATTN_E_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return ATTN_E_ALIGN;
+  if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_E_TOO_LARGE;
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -402,18 +421,9 @@ int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const att
                          uint32_t *skip_mask, unsigned long long *skip_counts,
                          attn_bf16 *out, float *lse,
                          void *workspace, size_t workspace_bytes, attn_stream_t stream) {
-  if (batch < 0 || num_pages < 0 || max_pages_per_seq < 0) return ATTN_E_SHAPE;
-  if (page_size != kPageSize) return ATTN_E_PAGE_SIZE;
-  if (h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || h_q / h_kv > kMaxGroup) return ATTN_E_HEADS;
-  if (d != 64 && d != 128) return ATTN_E_HEAD_DIM;
-  if (!isfinite(scale) || !(scale > 0.f)) return ATTN_E_SCALE;
-  int rc = check_threshold(skip_threshold);
+  int rc = check_decode_args(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages,
+                             max_pages_per_seq, page_size, h_q, h_kv, d, skip_threshold, scale, out);
   if (rc) return rc;
-  if (batch > 0 && (num_pages <= 0 || max_pages_per_seq <= 0)) return ATTN_E_SHAPE;
-  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return ATTN_E_NULL;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return ATTN_E_ALIGN;
-  if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_E_TOO_LARGE;
   const bool skip = skip_threshold > 0.f;
   // skip mode: two passes over the split schedule with a workspace, one
   // sequential split per (sequence, kv-head) without
@@ -536,12 +546,15 @@ int attn_paged_decode_static(const attn_bf16 *q, const attn_bf16 *k_cache, const
                              int num_pages, int max_pages_per_seq, int page_size, int h_q, int h_kv,
                              int d, float skip_threshold, float scale, attn_bf16 *out, float *lse,
                              attn_stream_t stream) {
-  if (batch < 0 || h_q < 1 || d < 1 || max_pages_per_seq < 0) return ATTN_E_SHAPE;
+  // the same argument checks (and error codes) as attn_paged_decode_ex
+  int rc = check_decode_args(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages,
+                             max_pages_per_seq, page_size, h_q, h_kv, d, skip_threshold, scale, out);
+  if (rc) return rc;
   const bool skip = skip_threshold > 0.f;
   if (!skip && attn_paged_decode_workspace_size(batch, h_q, d) > ATTN_STATIC_WORKSPACE_BYTES)
     return ATTN_E_TOO_LARGE;
   unsigned int *err = nullptr;
-  int rc = device_state(&err);
+  rc = device_state(&err);
   if (rc) return rc;
   void *scratch = nullptr;
   rc = static_scratch(&scratch);

@@ -73,7 +73,8 @@ struct PrefillParams {
   int qb_max, kt_max;           // ceil(max_q / 128), ceil(max_k / 32)
   float scale_log2, thr_log2;
   unsigned int *err;
-  int work_slot;                // work-claim counter of this launch (set by launch_prefill)
+  int work_slot;                // work-claim slot of this launch (set by launch_prefill)
+  uint32_t work_tag;            // nonzero tag of this launch in its slot (set by launch_prefill)
   // item order: 0 = query blocks outermost (heaviest causal block first, for
   // s_q = s_k); 1 = sequences outermost (all items that read one sequence's
   // K/V run together, for prefixes longer than the queries)

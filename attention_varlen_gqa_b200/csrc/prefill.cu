@@ -54,12 +54,17 @@ constexpr int kSchedConsumers = 4 * kNQ + 2;   // warps that read each claimed i
 // Sequences ranked for the sequence-major item order (batches of up to
 // kRankMax sequences; larger batches keep their own order).
 constexpr int kRankMax = 32;
-// Work-claim counters, one pair (next item, CTAs done) per launch slot; the
-// last CTA of a launch puts its pair back to zero.  Launches take slots in
-// turn, so up to kWorkSlots prefill launches may run at the same time on a
-// device.
+// Work-claim slots.  A slot's word is (launch tag << 32) | next claim number,
+// 0 when free.  Every CTA of a launch first takes the slot for its launch's
+// tag (compare-and-swap from 0, or finding the tag already there); a CTA that
+// finds another launch's tag waits, bounded, until that launch frees it.
+// Claims are plain atomic adds.  A launch makes exactly `items` claims (each
+// CTA claims until it draws a number past the items), so the claim that draws
+// items - 1 is its last and puts the word back to 0.  Launches take slots in
+// turn; two that meet on a slot therefore run one after the other's claims
+// instead of sharing a counter.
 constexpr int kWorkSlots = 64;
-__device__ unsigned int g_work[kWorkSlots][2];
+__device__ unsigned long long g_work[kWorkSlots];
 constexpr int kThreads = 384;                  // softmax warpgroups 0, 1; warpgroup 2: TMA, MMA, 2 idle
 // Register split: launched at 168 per thread (384 x 168 = 64 512), the
 // producer / MMA warpgroup gives back down to 120 and each softmax warpgroup
@@ -123,6 +128,26 @@ ATTN_DEVICE bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abo
   *abort_flag = 1;
   raise_error(err, ATTN_DEVERR_TIMEOUT);
   return false;
+}
+
+// Take work-claim slot `slot` for the launch tagged `tag` (see g_work).  False
+// (ATTN_DEVERR_BUSY raised) when another launch held it for longer than the
+// wait limit.
+ATTN_DEVICE bool acquire_slot(unsigned long long *slot, uint32_t tag, unsigned int *err) {
+  const unsigned long long mine = (unsigned long long)tag << 32;
+  uint64_t t0 = 0;
+  for (;;) {
+    const unsigned long long prev = atomicCAS(slot, 0ull, mine);
+    if (prev == 0ull || (uint32_t)(prev >> 32) == tag) return true;
+    const uint64_t now = globaltimer_ns();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > kWaitLimitNs) {
+      raise_error(err, ATTN_DEVERR_BUSY);
+      return false;
+    }
+    __nanosleep(1000);
+  }
 }
 
 ATTN_DEVICE void drain(uint64_t *bar, uint32_t parity) {
@@ -703,7 +728,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 0) {
-      unsigned int *next_item = &g_work[p.work_slot][0];
+      unsigned long long *slot = &g_work[p.work_slot];
+      const bool owned = acquire_slot(slot, p.work_tag, p.err);
+      // the next claimed item number; the launch's last claim frees the slot
+      auto claim = [&]() -> int {
+        const unsigned long long old = atomicAdd(slot, 1ull);
+        const uint32_t c = (uint32_t)old;
+        if ((uint32_t)(old >> 32) != p.work_tag) raise_error(p.err, ATTN_DEVERR_BUSY);
+        if (c + 1u == (uint32_t)items) atomicExch(slot, 0ull);
+        return (int)gridDim.x + (int)c;
+      };
       // an item holds work when one of its query tiles holds rows (a tile
       // whose rows see no key still writes zeros and -inf); items of a
       // sequence with broken cu_seqlens are reported and dropped here
@@ -719,18 +753,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < kNQ; ++t) any = any || tile_geo(p, sq, it.r[t]).active;
         return any;
       };
-      int next = (int)blockIdx.x;
+      // a CTA that could not take the slot does no work (the error is raised)
+      int next = owned ? (int)blockIdx.x : items;
       for (uint32_t n = 0;; ++n) {
-        while (next < items && !has_work(next)) next = (int)gridDim.x + (int)atomicAdd(next_item, 1u);
-        const uint32_t slot = n % kSchedDepth;
+        while (next < items && !has_work(next)) next = claim();
+        const uint32_t rs = n % kSchedDepth;
         if (n >= kSchedDepth &&
-            !wait_or_abort(&sched_empty[slot], ((n / kSchedDepth) - 1) & 1, abort_flag, p.err))
+            !wait_or_abort(&sched_empty[rs], ((n / kSchedDepth) - 1) & 1, abort_flag, p.err))
           break;
-        ring[slot] = next < items ? next : -1;
-        mbar_arrive(&sched_full[slot]);
+        ring[rs] = next < items ? next : -1;
+        mbar_arrive(&sched_full[rs]);
         if (next >= items) break;
-        next = (int)gridDim.x + (int)atomicAdd(next_item, 1u);
+        next = claim();
       }
+      // after an abort, the remaining claims are still drawn, so that the
+      // launch's count completes and the slot is freed
+      while (owned && next < items) next = claim();
     }
   }
   } else {
@@ -1000,23 +1038,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  // every claim of this CTA is made; the last CTA to get here rearms the slot
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(&g_work[p.work_slot][1], 1u) == gridDim.x - 1) {
-      atomicExch(&g_work[p.work_slot][0], 0u);
-      atomicExch(&g_work[p.work_slot][1], 0u);
-    }
-  }
 }
 
+// SM count of the current device, looked up once per device.
 int num_sms() {
-  static int n = 0;
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> count[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  if (dev >= kMaxDevices) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 1;
+  }
+  int n = count[dev].load(std::memory_order_relaxed);
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (n <= 0) n = 1;
+    count[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }
@@ -1031,9 +1070,11 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUte
   const long long items = (p.group % 2 == 0) ? (long long)p.batch * p.qb_max * (p.h_q / 2)
                                              : (long long)p.batch * ((p.qb_max + 1) / 2) * p.h_q;
   const int grid = (int)(items < num_sms() ? items : num_sms());
-  static std::atomic<unsigned int> next_slot{0};
+  // a nonzero tag per launch; launches take the claim slots in turn
+  static std::atomic<unsigned int> next_tag{0};
   PrefillParams q = p;
-  q.work_slot = (int)(next_slot.fetch_add(1u) % kWorkSlots);
+  q.work_tag = next_tag.fetch_add(1u) % 0xffffffffu + 1u;
+  q.work_slot = (int)(q.work_tag % kWorkSlots);
   prefill_kernel<D, SKIP><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, omap, q);
   return cudaGetLastError();
 }

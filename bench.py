@@ -36,6 +36,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -146,12 +147,12 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            fd, self.path = tempfile.mkstemp(prefix=f"clocks_rank{self.index}_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
@@ -180,6 +181,7 @@ class ClockSampler:
                 for n, v in zip(names, parts[5:9]):
                     if v.lower().startswith("active"):
                         reasons.add(n)
+        os.unlink(self.path)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
@@ -533,7 +535,8 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": agg["e2e_value"], "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": agg["e2e_ms"],
-                "what": "prefill through attn_varlen_fwd with q/k/v/cu_seqlens copied from pinned host "
+                "what": "prefill through the C entry point attn_varlen_fwd (the binding calls it when no "
+                        "skip threshold, mask or counts are asked for) with q/k/v/cu_seqlens copied from pinned host "
                         "memory and out/lse copied back every step; steps pipelined over two device "
                         "buffer sets (copy-in, kernel and read-back on three streams)"},
         "gpu_launches": 4 * args.steps,

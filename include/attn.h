@@ -93,7 +93,9 @@ enum attn_device_error {
   ATTN_DEVERR_SEQ_LEN = 1u << 1,     /* decode seq_len < 0 or > max_pages_per_seq*page    */
   ATTN_DEVERR_BLOCK_TABLE = 1u << 2, /* block-table entry outside [0, num_pages)          */
   ATTN_DEVERR_SMALLSEQ_LEN = 1u << 3,/* small-seq row with s_kv > max_s_kv                */
-  ATTN_DEVERR_TIMEOUT = 1u << 4      /* a pipeline wait gave up (kernel returned early)   */
+  ATTN_DEVERR_TIMEOUT = 1u << 4,     /* a pipeline wait gave up (kernel returned early)   */
+  ATTN_DEVERR_BUSY = 1u << 5         /* a prefill work-claim slot stayed held by another
+                                        launch past the wait limit (rows not written)    */
 };
 
 /* Compile-time tile geometry of this build (reported for the tests). */
@@ -129,11 +131,14 @@ ATTN_API const char *attn_status_string(int status);
  *
  * Work balance: the kernel's CTAs claim work items from a counter the library
  * keeps in device memory, one of 64 per device taken in turn by successive
- * calls (attn_varlen_fwd and attn_varlen_fwd_ex alike) and re-zeroed by the
- * kernel itself when it ends.  Up to 64 of these calls may therefore run
- * concurrently on one device (on different streams, or as parallel branches
- * of a CUDA graph); a 65th that overlaps them shares a counter and computes
- * wrong rows.
+ * launches (attn_varlen_fwd, attn_varlen_fwd_ex and attn_paged_prefill
+ * alike).  Each launch tags its counter and frees it with its last claim; a
+ * launch that meets a counter still held by another waits until it is freed
+ * (at most about one second), so any number of these calls may run
+ * concurrently on one device.  A wait that runs out sets ATTN_DEVERR_BUSY
+ * and the waiting part of the launch writes nothing.  Two concurrent replays
+ * of one captured CUDA graph share its launches' tags and must not overlap
+ * (they would also write the same outputs).
  *
  * Returns ATTN_OK or an ATTN_E_* code (nothing launched on error).
  */
@@ -203,7 +208,7 @@ ATTN_API int attn_varlen_fwd_ex(const attn_bf16 *q, const attn_bf16 *k, const at
  * entry outside [0, num_pages) sets ATTN_DEVERR_BLOCK_TABLE and that page is
  * read as zeros; a bad cu_seqlens_q or seq_lens_k entry sets
  * ATTN_DEVERR_CU_SEQLENS and the sequence is not written.  Shares the
- * work-claim counters of attn_varlen_fwd (64 concurrent calls per device).
+ * work-claim counters of attn_varlen_fwd (see there).
  */
 ATTN_API int attn_paged_prefill(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
                        const int32_t *block_table, const int32_t *cu_seqlens_q,
@@ -252,11 +257,19 @@ ATTN_API int attn_varlen_bwd(const attn_bf16 *q, const attn_bf16 *k, const attn_
  * needs for this shape (a pure host query; 0 is never returned for
  * batch * h_q > 0).  The dense schedule keeps, per (sequence, q-head, split),
  * the split's running max, running sum and unnormalised output in float32.
+ * The caller asks for the size first and passes a buffer of at least that
+ * many bytes, the shape- and workspace-query convention of
+ * ROCm/TransformerEngine PR 461 ("Integrate CK varlen cross attention for
+ * small-seq (s_q=1, s_kv<=16)", description bullets: the forward and
+ * backward each get a workspace-size query that the caller runs before the
+ * launch).  Sizes: 32 * batch * h_q * (4 d + 8) bytes, each of its two parts
+ * (outputs, then max and sum) rounded up to 256 bytes.
  */
 ATTN_API size_t attn_paged_decode_workspace_size(int batch, int h_q, int d);
 
 /*
- * attn_paged_decode_workspace_size_ex -- the same query for either schedule:
+ * attn_paged_decode_workspace_size_ex -- the same query (same convention,
+ * ROCm/TransformerEngine PR 461, description bullets) for either schedule:
  * skip_threshold == 0 gives attn_paged_decode_workspace_size(batch, h_q, d);
  * skip_threshold > 0 gives the two-pass skip schedule's need: the split
  * partials plus, in float32, the scores of every (query head, key slot up to
@@ -335,8 +348,10 @@ ATTN_API int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, 
  *
  *   - scratch limit: ATTN_STATIC_WORKSPACE_BYTES (48 MiB).  A dense-mode
  *     shape whose attn_paged_decode_workspace_size(batch, h_q, d) exceeds it
- *     returns ATTN_E_TOO_LARGE and launches nothing (about batch * h_q <=
- *     2900 at d = 128, <= 5600 at d = 64).  In skip mode the two-pass
+ *     returns ATTN_E_TOO_LARGE and launches nothing: the shape fits when
+ *     32 * batch * h_q * (4 d + 8) bytes, with the two parts (outputs, then
+ *     max and sum) each rounded up to 256, is at most 48 MiB, i.e.
+ *     batch * h_q <= 3024 at d = 128 and <= 5957 at d = 64.  In skip mode the two-pass
  *     schedule runs when its workspace fits the array, the sequential one
  *     (no workspace) otherwise.
  *   - every GPU that loads the library reserves those 48 MiB until the
@@ -351,6 +366,8 @@ ATTN_API int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, 
  *     it and give wrong results; order them on one stream or use
  *     attn_paged_decode with a workspace per stream.
  *   - no cudaMalloc, cudaFree or other allocating routine is called.
+ *   - argument errors are checked, and reported with the same codes, as by
+ *     attn_paged_decode_ex; ATTN_E_TOO_LARGE comes after those checks.
  */
 #define ATTN_STATIC_WORKSPACE_BYTES ((size_t)48 << 20)
 ATTN_API int attn_paged_decode_static(const attn_bf16 *q, const attn_bf16 *k_cache,

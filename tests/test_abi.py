@@ -222,3 +222,39 @@ def test_varlen_bwd_argument_errors(A):
     assert varlen_bwd(A, mk=1 << 25) == -13
     assert A.lib.attn_varlen_bwd_workspace_size(10, 4) == 256
     assert A.lib.attn_varlen_bwd_workspace_size(1000, 32) == 1000 * 32 * 4
+
+
+def static_decode(A, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, batch=2, pages=4, maxp=2, ps=16, hq=8, hkv=2, d=128,
+             thr=0.0, scale=0.1, out=FAKE, lse=None, stream=None)
+    a.update(kw)
+    return A.lib.attn_paged_decode_static(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["batch"], a["pages"],
+                                          a["maxp"], a["ps"], a["hq"], a["hkv"], a["d"], a["thr"], a["scale"],
+                                          a["out"], a["lse"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(ps=32), dict(hq=7), dict(hq=0), dict(hkv=0), dict(hq=64, hkv=2), dict(d=256), dict(d=0),
+    dict(thr=2.0), dict(thr=-1e-3), dict(thr=float("nan")), dict(scale=float("nan")), dict(scale=0.0),
+    dict(q=None), dict(kc=None), dict(vc=None), dict(bt=None), dict(sl=None), dict(out=None),
+    dict(q=FAKE + 8), dict(kc=FAKE + 2), dict(vc=FAKE + 4), dict(out=FAKE + 8), dict(pages=0), dict(maxp=0),
+    dict(batch=-1), dict(maxp=1 << 27)])
+def test_static_decode_argument_errors_match_workspace_entry(A, bad):
+    """attn_paged_decode_static checks its arguments like attn_paged_decode_ex
+    and returns the same codes (all before any CUDA call)."""
+    rc = static_decode(A, **bad)
+    assert rc < 0
+    assert rc == decode(A, **bad)
+
+
+def test_static_decode_too_large_after_argument_checks(A):
+    # batch * h_q = 3025 at d = 128 is one row over the 48 MiB scratch array
+    assert A.lib.attn_paged_decode_workspace_size(3024, 1, 128) <= 48 << 20
+    assert A.lib.attn_paged_decode_workspace_size(3025, 1, 128) > 48 << 20
+    assert A.lib.attn_paged_decode_workspace_size(5957, 1, 64) <= 48 << 20
+    assert A.lib.attn_paged_decode_workspace_size(5958, 1, 64) > 48 << 20
+    assert static_decode(A, batch=3025, hq=1, hkv=1) == -13
+    assert static_decode(A, batch=5958, hq=1, hkv=1, d=64) == -13
+    # a bad argument is reported as such even when the shape is too large
+    assert static_decode(A, batch=3025, hq=1, hkv=1, d=96) == -4
+    assert static_decode(A, batch=3025, hq=1, hkv=1, q=None) == -1

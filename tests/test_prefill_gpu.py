@@ -250,3 +250,33 @@ def test_concurrent_calls_and_counter_reuse(A):
     for o in again:
         assert torch.equal(o[0], r1[0]) and torch.equal(o[1], r1[1])
     assert A.attn_get_last_device_error() == 0
+
+
+def test_many_overlapping_calls_share_claim_slots(A):
+    """160 calls on four streams with no ordering between the streams, more
+    than the 64 work-claim slots: calls that meet on a slot take it in turn
+    (a launch tags its slot and frees it with its last claim), so every result
+    equals the single call's bit for bit and no error bit is raised."""
+    data = [W.varlen_prefill([300, 129, 64], h_q=8, h_kv=2, d=64, causal=True, seed=31),
+            W.varlen_prefill([1000, 17], h_q=4, h_kv=4, d=128, causal=False, seed=32),
+            W.varlen_prefill([513], h_q=16, h_kv=2, d=128, causal=True, seed=33),
+            W.varlen_prefill([40, 80, 120, 160], h_q=2, h_kv=1, d=64, causal=True, seed=34)]
+    devs = [_dev(d) for d in data]
+
+    def call(d, t):
+        return A.attn_varlen_fwd(t["q"], t["k"], t["v"], t["cu_q"], t["cu_k"], d["max_q"], d["max_k"],
+                                 causal=d["causal"], scale=d["scale"])
+
+    refs = [call(d, t) for d, t in zip(data, devs)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in data]
+    outs = [[] for _ in data]
+    for _ in range(40):
+        for i, (d, t) in enumerate(zip(data, devs)):
+            with torch.cuda.stream(streams[i]):
+                outs[i].append(call(d, t))
+    torch.cuda.synchronize()
+    assert A.attn_get_last_device_error() == 0
+    for ref, lst in zip(refs, outs):
+        for o in lst:
+            assert torch.equal(o[0], ref[0]) and torch.equal(o[1], ref[1])
