@@ -39,8 +39,6 @@ listed in the design notes):
 """
 from __future__ import annotations
 
-import math
-
 import numpy as np
 
 from .attention import NEG_INF, SkipRecord, bf16_bits_to_f64, gather_paged, kv_head_of, tile_decisions
