@@ -40,6 +40,8 @@ EXPORTS = {
     "attn_paged_decode": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _S, _P]),
     "attn_paged_decode_ex": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P, _P, _P, _S, _P]),
     "attn_paged_decode_static": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _P, _P, _P]),
+    "attn_paged_decode_qdq_workspace_size": (_S, [_I, _I, _I, _I]),
+    "attn_paged_decode_qdq": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _I, _F, _I, _F] + [_P] * 5 + [_S, _P]),
     "attn_paged_decode_workspace_size_ex": (_S, [_I, _I, _I, _I, _F]),
     "attn_smallseq_fwd": (_I, [_P] * 4 + [_I] * 5 + [_F, _P, _P, _P]),
     "attn_smallseq_bwd": (_I, [_P] * 6 + [_I] * 5 + [_F, _P, _P, _P, _P]),
@@ -220,14 +222,26 @@ def attn_paged_decode_workspace_size(batch, h_q, d, max_pages_per_seq=0, skip_th
     return int(lib.attn_paged_decode_workspace_size(batch, h_q, d))
 
 
+QDQ_FORMATS = {None: 0, "none": 0, "nvfp4": 1}
+
+
 def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size=16, skip_threshold=0.0,
                       scale=None, out=None, lse=None, workspace=None, skip_mask=None,
-                      skip_counts=None, want_lse=True, skip_schedule="split", stream=None):
+                      skip_counts=None, want_lse=True, skip_schedule="split", p_qdq=None, p_qdq_amax=1.0,
+                      v_qdq=None, v_qdq_amax=1.0, stream=None):
     """One-token paged decode. q [B, h_q, d]; caches [pages, page_size, h_kv, d];
     block_table int32 [B, max_pages]; seq_lens int32 [B].  Returns (out, lse).
-    skip_schedule (skip_threshold > 0): "split" -- two passes over the split
-    schedule with a workspace (allocated here when not given); "sequential" --
-    one split per (sequence, kv-head), no workspace."""
+    skip_schedule (skip_threshold > 0, or P / V quantised): "split" -- two
+    passes over the split schedule with a workspace (allocated here when not
+    given); "sequential" -- one split per (sequence, kv-head), no workspace.
+    p_qdq / v_qdq: None or "nvfp4" (NVFP4 quantise-dequantise of P / V before
+    their product, with the operand's amax)."""
+    if p_qdq not in QDQ_FORMATS or v_qdq not in QDQ_FORMATS:
+        raise ValueError(f"p_qdq / v_qdq must be one of {sorted(k for k in QDQ_FORMATS if k)} or None")
+    if QDQ_FORMATS[p_qdq] or QDQ_FORMATS[v_qdq]:
+        return _paged_decode_qdq(q, k_cache, v_cache, block_table, seq_lens, page_size, skip_threshold, scale,
+                                 out, lse, workspace, skip_mask, skip_counts, want_lse, skip_schedule,
+                                 QDQ_FORMATS[p_qdq], p_qdq_amax, QDQ_FORMATS[v_qdq], v_qdq_amax, stream)
     _need(q, "q", torch.bfloat16, 3)
     _need(k_cache, "k_cache", torch.bfloat16, 4)
     _need(v_cache, "v_cache", torch.bfloat16, 4)
@@ -265,6 +279,42 @@ def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size=16, 
             _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
             _stream(stream))
     _check("attn_paged_decode", rc)
+    return out, lse
+
+
+def _paged_decode_qdq(q, k_cache, v_cache, block_table, seq_lens, page_size, skip_threshold, scale, out, lse,
+                      workspace, skip_mask, skip_counts, want_lse, skip_schedule, p_fmt, p_amax, v_fmt, v_amax,
+                      stream):
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    batch, h_q, d = q.shape
+    num_pages, ps, h_kv, _ = k_cache.shape
+    if ps != page_size:
+        raise ValueError(f"cache page dimension {ps} != page_size {page_size}")
+    if skip_schedule not in ("split", "sequential"):
+        raise ValueError(f"skip_schedule must be 'split' or 'sequential', got {skip_schedule!r}")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((batch, h_q), dtype=torch.float32, device=q.device)
+    ws_bytes = 0
+    if skip_schedule == "sequential":
+        workspace = None
+    else:
+        need = int(lib.attn_paged_decode_qdq_workspace_size(batch, h_q, d, block_table.shape[1]))
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib.attn_paged_decode_qdq(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), batch, num_pages,
+        block_table.shape[1], page_size, h_q, h_kv, d, float(skip_threshold), scale, p_fmt, float(p_amax), v_fmt,
+        float(v_amax), _ptr(skip_mask), _ptr(skip_counts), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+        _stream(stream))
+    _check("attn_paged_decode_qdq", rc)
     return out, lse
 
 

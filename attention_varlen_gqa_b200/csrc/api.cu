@@ -129,6 +129,7 @@ const char *attn_status_string(int status) {
     case ATTN_E_CUDA: return "ATTN_E_CUDA";
     case ATTN_E_DEVICE: return "ATTN_E_DEVICE";
     case ATTN_E_TOO_LARGE: return "ATTN_E_TOO_LARGE";
+    case ATTN_E_QDQ: return "ATTN_E_QDQ";
     default: return "ATTN_E_UNKNOWN";
   }
 }
@@ -414,25 +415,43 @@ size_t attn_paged_decode_workspace_size_ex(int batch, int h_q, int d, int max_pa
   return skip_workspace(batch, h_q, d, max_pages_per_seq).total;
 }
 
-int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
-                         const int32_t *block_table, const int32_t *seq_lens,
-                         int batch, int num_pages, int max_pages_per_seq, int page_size,
-                         int h_q, int h_kv, int d, float skip_threshold, float scale,
-                         uint32_t *skip_mask, unsigned long long *skip_counts,
-                         attn_bf16 *out, float *lse,
-                         void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// NVFP4 quantise-dequantise of the decode's P and V (see attn.h).
+struct QdqSpec {
+  bool p, v;
+  float p_amax, v_amax;
+};
+
+// 448 / amax, and the ratio table g / (1 + j / 8), g = 2688 / amax (fp32).
+void qdq_constants(float amax, float *k, float *tab) {
+  *k = 448.0f / amax;
+  const float g = 2688.0f / amax;
+  for (int j = 0; j < 8; ++j) tab[j] = g / (1.0f + (float)j / 8.0f);
+}
+
+int paged_decode_impl(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                      const int32_t *block_table, const int32_t *seq_lens, int batch, int num_pages,
+                      int max_pages_per_seq, int page_size, int h_q, int h_kv, int d, float skip_threshold,
+                      float scale, const QdqSpec *qdq, uint32_t *skip_mask, unsigned long long *skip_counts,
+                      attn_bf16 *out, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream) {
   int rc = check_decode_args(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages,
                              max_pages_per_seq, page_size, h_q, h_kv, d, skip_threshold, scale, out);
   if (rc) return rc;
-  const bool skip = skip_threshold > 0.f;
+  const bool quant = qdq && (qdq->p || qdq->v);
+  // the 32-key skip schedules: skip-softmax on, or P / V quantised (at any threshold)
+  const bool skip = skip_threshold > 0.f || quant;
   // skip mode: two passes over the split schedule with a workspace, one
   // sequential split per (sequence, kv-head) without
   const bool two_pass = skip && workspace != nullptr;
   if ((!skip || two_pass) && batch > 0) {
     if (!workspace) return ATTN_E_WORKSPACE;
     if (!aligned16(workspace)) return ATTN_E_ALIGN;
-    if (workspace_bytes < attn_paged_decode_workspace_size_ex(batch, h_q, d, max_pages_per_seq, skip_threshold))
-      return ATTN_E_WORKSPACE;
+    const size_t need = skip ? skip_workspace(batch, h_q, d, max_pages_per_seq).total
+                             : attn_paged_decode_workspace_size(batch, h_q, d);
+    if (workspace_bytes < need) return ATTN_E_WORKSPACE;
   }
   unsigned int *err = nullptr;
   rc = device_state(&err);
@@ -463,6 +482,20 @@ int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const att
   p.scale_log2 = scale * 1.4426950408889634f;
   p.thr_log2 = thr_to_log2(skip_threshold);
   p.sequential = skip ? (two_pass ? 2 : 1) : 0;
+  if (quant) {
+    p.p_qdq = qdq->p ? 1 : 0;
+    p.v_qdq = qdq->v ? 1 : 0;
+    float inv = 1.0f;
+    if (qdq->p) {
+      qdq_constants(qdq->p_amax, &p.p_k, p.p_tab);
+      inv *= qdq->p_amax / 2688.0f;
+    }
+    if (qdq->v) {
+      qdq_constants(qdq->v_amax, &p.v_k, p.v_tab);
+      inv *= qdq->v_amax / 2688.0f;
+    }
+    p.qdq_out = inv;
+  }
   if (two_pass && batch > 0) {
     const SkipWorkspace w = skip_workspace(batch, h_q, d, max_pages_per_seq);
     char *base = static_cast<char *>(workspace);
@@ -490,6 +523,46 @@ int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const att
       encode_3d(&vmap, v_cache, d, h_kv, slots, kPageSize))
     return ATTN_E_CUDA;
   return launch_decode(p, kmap, vmap, st) == cudaSuccess ? ATTN_OK : ATTN_E_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                         const int32_t *block_table, const int32_t *seq_lens,
+                         int batch, int num_pages, int max_pages_per_seq, int page_size,
+                         int h_q, int h_kv, int d, float skip_threshold, float scale,
+                         uint32_t *skip_mask, unsigned long long *skip_counts,
+                         attn_bf16 *out, float *lse,
+                         void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  return paged_decode_impl(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages, max_pages_per_seq,
+                           page_size, h_q, h_kv, d, skip_threshold, scale, nullptr, skip_mask, skip_counts, out,
+                           lse, workspace, workspace_bytes, stream);
+}
+
+size_t attn_paged_decode_qdq_workspace_size(int batch, int h_q, int d, int max_pages_per_seq) {
+  return attn_paged_decode_workspace_size_ex(batch, h_q, d, max_pages_per_seq, 1.0f);
+}
+
+int attn_paged_decode_qdq(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                          const int32_t *block_table, const int32_t *seq_lens, int batch, int num_pages,
+                          int max_pages_per_seq, int page_size, int h_q, int h_kv, int d, float skip_threshold,
+                          float scale, int p_qdq, float p_qdq_amax, int v_qdq, float v_qdq_amax,
+                          uint32_t *skip_mask, unsigned long long *skip_counts, attn_bf16 *out, float *lse,
+                          void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  int rc = check_decode_args(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages, max_pages_per_seq,
+                             page_size, h_q, h_kv, d, skip_threshold, scale, out);
+  if (rc) return rc;
+  auto amax_ok = [](float a) { return isfinite(a) && a >= 0x1p-64f && a <= 0x1p64f; };
+  if ((p_qdq != ATTN_QDQ_NONE && p_qdq != ATTN_QDQ_NVFP4) || (v_qdq != ATTN_QDQ_NONE && v_qdq != ATTN_QDQ_NVFP4))
+    return ATTN_E_QDQ;
+  if ((p_qdq == ATTN_QDQ_NVFP4 && !amax_ok(p_qdq_amax)) || (v_qdq == ATTN_QDQ_NVFP4 && !amax_ok(v_qdq_amax)))
+    return ATTN_E_QDQ;
+  QdqSpec spec{p_qdq == ATTN_QDQ_NVFP4, v_qdq == ATTN_QDQ_NVFP4, p_qdq_amax, v_qdq_amax};
+  return paged_decode_impl(q, k_cache, v_cache, block_table, seq_lens, batch, num_pages, max_pages_per_seq,
+                           page_size, h_q, h_kv, d, skip_threshold, scale, &spec, skip_mask, skip_counts, out,
+                           lse, workspace, workspace_bytes, stream);
 }
 
 int attn_paged_decode(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,

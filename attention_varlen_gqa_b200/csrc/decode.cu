@@ -38,6 +38,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "nvfp4.cuh"
 
 namespace attn {
 namespace {
@@ -65,7 +66,9 @@ struct DecodeLayout {
   static constexpr int kK = 0;
   static constexpr int kS = SEQ ? kSeqSlots * kSlot : 2 * kDenseStages * kSlot;
   static constexpr int kQmax = kS + (SEQ ? kSeqRing * kWarps * 32 * kRingFloats * 4 : 0);
-  static constexpr int kBar = kQmax + (SEQ ? 2 * kWarps * 16 * 4 : 0);
+  // sequential: the walk's running max after each tile, [ring][tile][head] (QDQ)
+  static constexpr int kMrun = kQmax + (SEQ ? 2 * kWarps * 16 * 4 : 0);
+  static constexpr int kBar = kMrun + (SEQ ? kSeqRing * 2 * kMaxGroup * 4 : 0);
   static constexpr int kNumBars = SEQ ? 2 * kSeqSlots : kDenseStages;
   static constexpr int kBt = kBar + kNumBars * 8;                  // the CTA's block-table entries
   static constexpr int kBtCap = SEQ ? 2048 : 256;                  // entries (longer ranges read global)
@@ -223,6 +226,112 @@ ATTN_DEVICE void warp_pv(float (&o_acc)[D / 16][NH][4], float (&m_w)[NH][2], flo
   }
 }
 
+// The lane's entry of a QDQ ratio table (lane j holds entry j & 7).
+ATTN_DEVICE float table_entry(const float (&tab)[8], int lane) {
+  float t = tab[0];
+#pragma unroll
+  for (int j = 1; j < 8; ++j)
+    if ((lane & 7) == j) t = tab[j];
+  return t;
+}
+
+// warp_pv with NVFP4 quantise-dequantise of P and / or V.  Every warp takes
+// as its reference max the running max of the 32-key walk after this tile,
+// mt[n][h] (heads 8 n + cq + h; the same for every warp), so that p =
+// exp(s - M_t) as the walk defines it; l sums the unquantised p.  A warp's 16
+// tokens are one page, so a P block is one head's 16 p of this warp (8 lanes
+// x 2) and a V block one channel's 16 values (4 lanes x 4).  With V quantised
+// the P V MMAs take f16 operands (the dequantised products q * s are exact in
+// f16), else bf16; O accumulates in units of g_p g_v (p.qdq_out undoes it).
+template <int D, int NH>
+ATTN_DEVICE void warp_pv_qdq(float (&o_acc)[D / 16][NH][4], float (&m_w)[NH][2], float (&l_w)[NH][2],
+                             const float (&s)[NH][4], const float (&mt)[NH][2], uint32_t vslot, const Lane &ln,
+                             const DecodeParams &p, float p_tab, float v_tab) {
+  float alpha[NH][2];
+  bool rescale = false;
+#pragma unroll
+  for (int n = 0; n < NH; ++n)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float m_new = fmaxf(m_w[n][h], mt[n][h]);
+      alpha[n][h] = (m_w[n][h] == -INFINITY) ? 0.f : ex2(m_w[n][h] - m_new);
+      m_w[n][h] = m_new;
+      l_w[n][h] *= alpha[n][h];
+      rescale |= alpha[n][h] != 1.f;
+    }
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int n = 0; n < NH; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o_acc[t][n][e] *= alpha[n][e & 1];
+  }
+  const bool vq = p.v_qdq != 0;
+  uint32_t pb[NH][2];
+#pragma unroll
+  for (int n = 0; n < NH; ++n) {
+    const float mr0 = (m_w[n][0] == -INFINITY) ? 0.f : m_w[n][0];
+    const float mr1 = (m_w[n][1] == -INFINITY) ? 0.f : m_w[n][1];
+    const float p0 = ex2(s[n][0] - mr0), p1 = ex2(s[n][1] - mr1);   // token g, heads cq, cq + 1
+    const float p2 = ex2(s[n][2] - mr0), p3 = ex2(s[n][3] - mr1);   // token g + 8
+    l_w[n][0] += p0 + p2;
+    l_w[n][1] += p1 + p3;
+    uint32_t x01, x23;                                               // f16x2 operand pairs
+    if (p.p_qdq) {
+      // block max of heads cq, cq + 1 over the warp's 16 tokens (lanes g = 0..7)
+      float b0 = fmaxf(p0, p2), b1 = fmaxf(p1, p3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, o));
+        b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, o));
+      }
+      const uint32_t sc = e4m3x2_as_f16x2(__fmul_rn(b0, p.p_k), __fmul_rn(b1, p.p_k));
+      const float r0 = ratio_from_table(f16_lo(sc), p_tab), r1 = ratio_from_table(f16_hi(sc), p_tab);
+      x01 = hmul2_u32(e2m1x2_as_f16x2(__fmul_rn(p0, r0), __fmul_rn(p1, r1)), sc);
+      x23 = hmul2_u32(e2m1x2_as_f16x2(__fmul_rn(p2, r0), __fmul_rn(p3, r1)), sc);
+      if (!vq) {
+        x01 = f16x2_to_bf16x2(x01);
+        x23 = f16x2_to_bf16x2(x23);
+      }
+    } else if (vq) {
+      x01 = pack_f16x2(p0, p1);
+      x23 = pack_f16x2(p2, p3);
+    } else {
+      x01 = pack_bf16x2(p0, p1);
+      x23 = pack_bf16x2(p2, p3);
+    }
+    pb[n][0] = movmatrix_trans(x01);
+    pb[n][1] = movmatrix_trans(x23);
+  }
+  const int tok = ln.w * 16 + (ln.lane & 7) + ((ln.lane >> 4) & 1) * 8;
+#pragma unroll
+  for (int mt_ = 0; mt_ < D / 16; ++mt_) {
+    uint32_t a[4];
+    ldsm_x4_trans(slot_addr(vslot, tok, 2 * mt_ + ((ln.lane >> 3) & 1)), a[0], a[1], a[2], a[3]);
+    if (vq) {
+      // a[0], a[2]: channel g of the m-tile, tokens 2 (lane % 4) + {0, 1} and
+      // + 8; a[1], a[3]: channel g + 8.  Block max over the 4 lanes of a row.
+      uint32_t bm = absmax_pairs_bf16(a[0], a[2], a[1], a[3]);
+      bm = max_bf16x2(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = max_bf16x2(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+      const uint32_t sc = e4m3x2_as_f16x2(__fmul_rn(bf16_lo(bm), p.v_k), __fmul_rn(bf16_hi(bm), p.v_k));
+      const float r_g = ratio_from_table(f16_lo(sc), v_tab), r_g8 = ratio_from_table(f16_hi(sc), v_tab);
+      const uint32_t s_g = f16x2_bcast(sc, false), s_g8 = f16x2_bcast(sc, true);
+      uint32_t f[4];
+      f[0] = qdq_bf16_pair(a[0], r_g, s_g);
+      f[1] = qdq_bf16_pair(a[1], r_g8, s_g8);
+      f[2] = qdq_bf16_pair(a[2], r_g, s_g);
+      f[3] = qdq_bf16_pair(a[3], r_g8, s_g8);
+#pragma unroll
+      for (int n = 0; n < NH; ++n) mma_f16_16816(o_acc[mt_][n], f, pb[n][0], pb[n][1]);
+    } else {
+#pragma unroll
+      for (int n = 0; n < NH; ++n) mma_bf16_16816(o_acc[mt_][n], a, pb[n][0], pb[n][1]);
+    }
+  }
+}
+
 // Merge the four warps' (m, l, O) and write the CTA's result: the split
 // partial (dense) or the normalised output and LSE (sequential).
 template <int D, int NH>
@@ -305,10 +414,11 @@ ATTN_DEVICE void issue_pages(const CUtensorMap *map, uint8_t *slot, uint64_t *ba
   }
 }
 
-template <int D, bool SEQ, int NH>
+template <int D, bool SEQ, int NH, bool QDQ>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           DecodeParams p) {
+  static_assert(SEQ || !QDQ, "quantise-dequantise runs in the skip schedules only");
   using Lay = DecodeLayout<D, SEQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = align1024(smem_raw);
@@ -427,6 +537,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       uint64_t *vfull = bars + kSeqSlots;             // [slot]: its kept V pages arrived
       float *s_ring = reinterpret_cast<float *>(base + Lay::kS);
       float *qmax = reinterpret_cast<float *>(base + Lay::kQmax);
+      float *mrun = reinterpret_cast<float *>(base + Lay::kMrun);   // [ring][tile][head]
+      float p_tab = 0.f, v_tab = 0.f;
+      if constexpr (QDQ) {
+        p_tab = table_entry(p.p_tab, ln.lane);
+        v_tab = table_entry(p.v_tab, ln.lane);
+      }
       auto slot_ptr = [&](int c) { return base + Lay::kK + (c % kSeqSlots) * Lay::kSlot; };
       int k_issued = 0, v_issued = 0;                 // chunks whose K / V copies were issued
       if (tid == 0)
@@ -483,6 +599,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             const bool vote = !head || (tm == -INFINITY) || (tm - m_run < p.thr_log2);
             m_run = fmaxf(m_run, tm);
             keep[tt] = !__all_sync(0xffffffffu, vote);
+            if (QDQ && ln.w == 0 && head) mrun[((i % kSeqRing) * 2 + tt) * kMaxGroup + ln.lane] = m_run;
           }
           if (!vis_b) keep[1] = false;
           if (tid == 0) {
@@ -528,7 +645,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 qm[nn][0] = sr[8 + 2 * nn];
                 qm[nn][1] = sr[9 + 2 * nn];
               }
-              warp_pv<D, NH>(o_acc, m_w, l_w, sv, qm, vslot, ln);
+              if constexpr (QDQ) {
+                // the walk's running max after this warp's tile (warps 0-1: tile A, 2-3: tile B)
+                const float *mr = mrun + ((j % kSeqRing) * 2 + (ln.w >> 1)) * kMaxGroup;
+#pragma unroll
+                for (int nn = 0; nn < NH; ++nn)
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const int hh = 8 * nn + ln.cq + h;
+                    qm[nn][h] = hh < G ? mr[hh] : -INFINITY;
+                  }
+                warp_pv_qdq<D, NH>(o_acc, m_w, l_w, sv, qm, vslot, ln, p, p_tab, v_tab);
+              } else {
+                warp_pv<D, NH>(o_acc, m_w, l_w, sv, qm, vslot, ln);
+              }
             }
           }
           // every warp is done with slot j % kSeqSlots: it takes the K of chunk j + kSeqSlots
@@ -557,6 +687,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       atomicAdd(p.skip_counts + 1, n_skip);
     }
     __syncthreads();
+  }
+  if constexpr (QDQ) {
+    // O was accumulated in units of g over the quantised operands
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int nn = 0; nn < NH; ++nn)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o_acc[t][nn][e] *= p.qdq_out;
   }
   merge_and_store<D, NH>(base + Lay::kK, o_acc, m_w, l_w, any_bad || failed, G, b, hk, split, nsplit, SEQ, p,
                      ln);
@@ -598,7 +737,9 @@ struct PassLayout {
   static constexpr int kTmax = kX + kDecodeSplits * kMaxGroup * 4;   // pass 2: the split's tile maxima
   // pass 2: per stage the chunk's decision bits, then per stage its chunk index
   static constexpr int kKeep = kTmax + (PV ? kTmaxCap * 4 : 0);
-  static constexpr int kBar = kKeep + 8 * kStages;
+  // pass 2: per stage the walk's running max after each of the chunk's tiles, [stage][tile][head] (QDQ)
+  static constexpr int kMrun = kKeep + 8 * kStages;
+  static constexpr int kBar = kMrun + (PV ? kStages * 2 * kMaxGroup * 4 : 0);
   static constexpr int kBt = kBar + kStages * 8;
   static constexpr int kBtCap = 256;
   static constexpr int kEnd = kBt + kBtCap * 4;
@@ -735,7 +876,7 @@ __global__ void __launch_bounds__(kThreads) decode_scores_kernel(const __grid_co
   }
 }
 
-template <int D, int NH>
+template <int D, int NH, bool QDQ>
 __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_constant__ CUtensorMap vmap,
                                                                   DecodeParams p) {
   using Lay = PassLayout<D, true>;
@@ -745,6 +886,7 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
   uint64_t *full = reinterpret_cast<uint64_t *>(base + Lay::kBar);
   float *tm_s = reinterpret_cast<float *>(base + Lay::kTmax);
   uint32_t *keep_s = reinterpret_cast<uint32_t *>(base + Lay::kKeep);
+  float *mrun_s = reinterpret_cast<float *>(base + Lay::kMrun);   // [stage][tile][head]
   const int tid = threadIdx.x;
   const Lane ln(tid);
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -793,11 +935,19 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
     }
     // warp 0 takes the decisions (lane h: head h) and issues the copies
     const bool head = ln.lane < G;
+    float p_tab = 0.f, v_tab = 0.f;
+    if constexpr (QDQ) {
+      p_tab = table_entry(p.p_tab, ln.lane);
+      v_tab = table_entry(p.v_tab, ln.lane);
+    }
     float m_run = -INFINITY;   // head lane's running max entering the next tile
     unsigned long long n_vis = 0, n_skip = 0;
     if (ln.w == 0 && head)
       for (int s2 = 0; s2 < split; ++s2) m_run = fmaxf(m_run, sm_s[s2 * G + ln.lane]);
     __syncthreads();   // barrier init
+    // decide() leaves the head lane's running max after each of the chunk's
+    // tiles in dm[] (the reference max of the quantised P)
+    float dm[2] = {-INFINITY, -INFINITY};
     auto decide = [&](int c) -> uint32_t {
       uint32_t kb = 0;
 #pragma unroll
@@ -810,6 +960,7 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
         // a head votes skip when exp(tile max - running max) < threshold
         const bool vote = !head || tm == -INFINITY || (tm - m_run < p.thr_log2);
         m_run = fmaxf(m_run, tm);
+        dm[tt] = m_run;
         const bool kept = vis && !__all_sync(0xffffffffu, vote);
         if (kept) kb |= 1u << tt;
         if (vis) {
@@ -849,6 +1000,7 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
     int next_c = 0;              // warp 0: the next chunk to decide
     int pend_c = 0;              // warp 0: the next kept chunk and its tile bits (0: none)
     uint32_t pend_kb = 0;
+    float pend_m[2] = {-INFINITY, -INFINITY};   // and its running maxima (QDQ)
     bool more = true;            // warp 0: the last entry is not issued yet
     auto find_kept = [&]() {
       pend_kb = 0;
@@ -856,10 +1008,19 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
         pend_c = next_c++;
         pend_kb = decide(pend_c);
       }
+      pend_m[0] = dm[0];
+      pend_m[1] = dm[1];
     };
     auto next_issue = [&](int i) {   // warp 0: ring position i
       const int c = pend_c;
       const uint32_t kb = pend_kb;
+      if constexpr (QDQ) {
+        if (kb && head) {
+          mrun_s[((i % Lay::kStages) * 2 + 0) * kMaxGroup + ln.lane] = pend_m[0];
+          mrun_s[((i % Lay::kStages) * 2 + 1) * kMaxGroup + ln.lane] = pend_m[1];
+        }
+        __syncwarp();
+      }
       if (kb) find_kept();
       if (ln.lane == 0) {
         if (kb) {
@@ -899,14 +1060,29 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
               sc[nn][e] = v;
               qm[nn][e & 1] = fmaxf(qm[nn][e & 1], v);
             }
+            if constexpr (!QDQ) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+              for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int o = 4; o < 32; o <<= 1)
-                qm[nn][h] = fmaxf(qm[nn][h], __shfl_xor_sync(0xffffffffu, qm[nn][h], o));
+                for (int o = 4; o < 32; o <<= 1)
+                  qm[nn][h] = fmaxf(qm[nn][h], __shfl_xor_sync(0xffffffffu, qm[nn][h], o));
+            }
           }
           zero_tail_rows<D>(base, vslot, tok_base, r.L, ln);
-          warp_pv<D, NH>(o_acc, m_w, l_w, sc, qm, vslot, ln);
+          if constexpr (QDQ) {
+            // the walk's running max after this warp's tile (warps 0-1: tile A, 2-3: tile B)
+            const float *mr = mrun_s + (s * 2 + (ln.w >> 1)) * kMaxGroup;
+#pragma unroll
+            for (int nn = 0; nn < NH; ++nn)
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int hh = 8 * nn + ln.cq + h;
+                qm[nn][h] = hh < G ? mr[hh] : -INFINITY;
+              }
+            warp_pv_qdq<D, NH>(o_acc, m_w, l_w, sc, qm, vslot, ln, p, p_tab, v_tab);
+          } else {
+            warp_pv<D, NH>(o_acc, m_w, l_w, sc, qm, vslot, ln);
+          }
         }
       }
       if (__syncthreads_or(!ok)) {
@@ -928,6 +1104,15 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
       atomicAdd(p.skip_counts + 1, n_skip);
     }
     __syncthreads();
+  }
+  if constexpr (QDQ) {
+    // O was accumulated in units of g over the quantised operands
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int nn = 0; nn < NH; ++nn)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o_acc[t][nn][e] *= p.qdq_out;
   }
   merge_and_store<D, NH>(base, o_acc, m_w, l_w, r.dead || failed, G, b, hk, split, kDecodeSplits, false, p,
                          ln);
@@ -965,48 +1150,59 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   if (p.lse && lane == 0) p.lse[row] = live ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
 }
 
-template <int D, bool SEQ, int NH>
+template <int D, bool SEQ, int NH, bool QDQ>
 cudaError_t launch_k(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
   const size_t smem = DecodeLayout<D, SEQ>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, SEQ, NH>,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, SEQ, NH, QDQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(SEQ ? 1 : kDecodeSplits, p.h_kv, p.batch);
-  decode_kernel<D, SEQ, NH><<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
+  decode_kernel<D, SEQ, NH, QDQ><<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
   return cudaGetLastError();
 }
 
 // one n-tile of 8 heads for groups of up to 8 query heads, two up to 16
-template <int D, bool SEQ>
+template <int D, bool SEQ, bool QDQ>
 cudaError_t launch_g(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
-  return p.group <= 8 ? launch_k<D, SEQ, 1>(p, kmap, vmap, stream) : launch_k<D, SEQ, 2>(p, kmap, vmap, stream);
+  return p.group <= 8 ? launch_k<D, SEQ, 1, QDQ>(p, kmap, vmap, stream)
+                      : launch_k<D, SEQ, 2, QDQ>(p, kmap, vmap, stream);
 }
 
-template <int D, int NH>
+template <int D, int NH, bool QDQ>
 cudaError_t launch_two_pass(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                             cudaStream_t stream) {
   const size_t s1 = PassLayout<D, false>::kBytes, s2 = PassLayout<D, true>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(decode_scores_kernel<D, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)s1);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_skip_pv_kernel<D, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
+  e = cudaFuncSetAttribute(decode_skip_pv_kernel<D, NH, QDQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)s2);
   if (e != cudaSuccess) return e;
   dim3 grid(kDecodeSplits, p.h_kv, p.batch);
   decode_scores_kernel<D, NH><<<grid, kThreads, s1, stream>>>(kmap, p);
-  decode_skip_pv_kernel<D, NH><<<grid, kThreads, s2, stream>>>(vmap, p);
+  decode_skip_pv_kernel<D, NH, QDQ><<<grid, kThreads, s2, stream>>>(vmap, p);
   return cudaGetLastError();
+}
+
+template <int D, bool QDQ>
+cudaError_t launch_two_pass_g(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                              cudaStream_t stream) {
+  return p.group <= 8 ? launch_two_pass<D, 1, QDQ>(p, kmap, vmap, stream)
+                      : launch_two_pass<D, 2, QDQ>(p, kmap, vmap, stream);
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
-  if (p.sequential == 1) return launch_g<D, true>(p, kmap, vmap, stream);
+  const bool qdq = p.p_qdq || p.v_qdq;
+  if (p.sequential == 1)
+    return qdq ? launch_g<D, true, true>(p, kmap, vmap, stream) : launch_g<D, true, false>(p, kmap, vmap, stream);
   cudaError_t e = p.sequential == 2
-                      ? (p.group <= 8 ? launch_two_pass<D, 1>(p, kmap, vmap, stream)
-                                      : launch_two_pass<D, 2>(p, kmap, vmap, stream))
-                      : launch_g<D, false>(p, kmap, vmap, stream);
+                      ? (qdq ? launch_two_pass_g<D, true>(p, kmap, vmap, stream)
+                             : launch_two_pass_g<D, false>(p, kmap, vmap, stream))
+                      : launch_g<D, false, false>(p, kmap, vmap, stream);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)p.batch * p.h_q;
   decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);

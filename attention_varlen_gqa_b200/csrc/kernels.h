@@ -60,6 +60,14 @@ struct DecodeParams {
   float scale_log2;             // scale * log2(e)
   float thr_log2;               // log2(threshold); -inf when skipping is off
   int sequential;               // skip mode: 1 = one split walking 32-key tiles, 2 = two passes
+  // NVFP4 quantise-dequantise of P and / or V (skip schedules only): which
+  // operands, their 448 / amax, their ratio tables g / (1 + j / 8), j = 0..7
+  // (g = 2688 / amax, fp32), and the output factor 1 / g over the quantised
+  // operands
+  int p_qdq, v_qdq;
+  float p_k, v_k;
+  float p_tab[8], v_tab[8];
+  float qdq_out;
   unsigned int *err;
 };
 

@@ -353,7 +353,7 @@ def main():
         assert A.attn_get_last_device_error() == 0
         return
     if args.only == "skip":
-        measure_skip(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
+        print(json.dumps(measure_skip(A, W, torch, dev, seed, pk, reps=max(1, args.steps))), flush=True)
         return
     if args.only == "paged_prefill":
         measure_paged_prefill(A, W, torch, dev, seed, pk, reps=max(1, args.steps))
@@ -582,7 +582,8 @@ def _skip_prefill_sweep(A, torch, dev, sp, reps, thresholds):
 
 
 def _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs):
-    """runs: (key, threshold, schedule) triples."""
+    """runs: (key, threshold, schedule) triples, or (key, threshold, schedule,
+    (p_amax, v_amax)) with NVFP4 quantise-dequantise of P and V."""
     import numpy as np
     bt = torch.from_numpy(sd["block_table"]).to(dev)
     sl = torch.from_numpy(sd["seq_lens"]).to(dev)
@@ -593,15 +594,19 @@ def _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs):
     counts = torch.zeros(2, dtype=torch.int64, device=dev)
     kbytes = float(sd["seq_lens"].astype(np.int64).sum() * h_kv * d * 2)
     res = {}
-    for key, thr, sched in runs:
+    for run_spec in runs:
+        key, thr, sched = run_spec[:3]
+        qdq = run_spec[3] if len(run_spec) > 3 else None
+        qkw = {} if qdq is None else dict(p_qdq="nvfp4", p_qdq_amax=qdq[0], v_qdq="nvfp4", v_qdq_amax=qdq[1])
         ws = None
         if sched == "split":
-            ws = torch.empty(A.attn_paged_decode_workspace_size(B, h_q, d, bt.shape[1], thr), dtype=torch.uint8,
-                             device=dev)
+            need = (A.lib.attn_paged_decode_qdq_workspace_size(B, h_q, d, bt.shape[1]) if qdq else
+                    A.attn_paged_decode_workspace_size(B, h_q, d, bt.shape[1], thr))
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
 
         def run():
             A.attn_paged_decode(sd["q"], sd["k_cache"], sd["v_cache"], bt, sl, skip_threshold=thr,
-                                out=out, lse=lse, workspace=ws, skip_counts=counts, skip_schedule=sched)
+                                out=out, lse=lse, workspace=ws, skip_counts=counts, skip_schedule=sched, **qkw)
         ms = _time_ms(torch, run, reps)
         vis, sk = (int(x) for x in counts.tolist())
         frac = sk / vis if vis and thr > 0 else 0.0
@@ -609,8 +614,10 @@ def _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs):
         alg = kbytes + kbytes * (1.0 - frac) + B * h_q * d * 2 * 2 + B * h_q * 4
         res[str(key)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
                          "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"],
-                         "schedule": "dense split-KV" if thr == 0 else
+                         "schedule": "dense split-KV" if thr == 0 and not qdq else
                          ("two passes over 32 splits" if sched == "split" else "one sequential split")}
+        if qdq:
+            res[str(key)]["qdq"] = f"NVFP4 P (amax {qdq[0]}) and V (amax {qdq[1]})"
     return res
 
 
@@ -622,6 +629,9 @@ def measure_skip(A, W, torch, dev, seed, pk, reps=3):
     # skip mode runs the two-pass schedule (workspace given); "0.1/sequential"
     # is the one-split-per-(sequence, kv-head) schedule at the same threshold
     runs = [(t, t, "split") for t in thresholds] + [("0.1/sequential", 0.1, "sequential")]
+    # NVFP4 quantise-dequantise of P and V (amax 1 each, the page's usage example)
+    runs += [(f"qdq/{t}", t, "split", (1.0, 1.0)) for t in thresholds]
+    runs += [("qdq/0.1/sequential", 0.1, "sequential", (1.0, 1.0))]
     res = {}
     sp = W.skip_prefill(seed=seed, where="device")
     res["prefill"] = _skip_prefill_sweep(A, torch, dev, sp, reps, thresholds)

@@ -84,7 +84,14 @@ enum attn_status {
   ATTN_E_SCALE = -10,      /* scale not finite or not > 0                        */
   ATTN_E_CUDA = -11,       /* a CUDA call failed (launch, tensor-map encode ...) */
   ATTN_E_DEVICE = -12,     /* current device is not compute capability 10.x      */
-  ATTN_E_TOO_LARGE = -13   /* a size exceeds a documented implementation limit   */
+  ATTN_E_TOO_LARGE = -13,  /* a size exceeds a documented implementation limit   */
+  ATTN_E_QDQ = -14         /* unknown QDQ format, or amax outside [2^-64, 2^64]  */
+};
+
+/* Quantise-dequantise formats of attn_paged_decode_qdq. */
+enum attn_qdq_format {
+  ATTN_QDQ_NONE = 0,       /* the operand stays as it is                         */
+  ATTN_QDQ_NVFP4 = 1       /* NVFP4: E2M1 values, E4M3 scales per 16, fp32 amax  */
 };
 
 /* Bits of the per-device error word. */
@@ -332,6 +339,48 @@ ATTN_API int attn_paged_decode_ex(const attn_bf16 *q, const attn_bf16 *k_cache, 
                          uint32_t *skip_mask, unsigned long long *skip_counts,
                          attn_bf16 *out, float *lse,
                          void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_paged_decode_qdq -- attn_paged_decode_ex with NVFP4 quantise-dequantise
+ * (QDQ) of the probabilities P and / or the values V before their product
+ * (NVIDIA/Model-Optimizer PR 1941, "Add split-k decode kernel for skip
+ * softmax", What does this PR do?, third bullet: skip-softmax together with
+ * NVFP4 P/V QDQ; Usage: p_qdq="nvfp4", p_qdq_amax, v_qdq="nvfp4",
+ * v_qdq_amax).  The page prints no recipe; this library's reading:
+ *
+ *   - blocks of 16 along the key axis (the contraction axis of P V): P per
+ *     query head over 16 consecutive keys, V per channel over 16 consecutive
+ *     keys (one page) of each kv-head;
+ *   - per block, with k = 448 / amax and g = 2688 / amax (fp32): s =
+ *     E4M3(max|x| * k), q = E2M1(x * (g / s)) (both round to nearest even and
+ *     saturate), dequantised value q * s / g; the code-deciding products and
+ *     the quotient g / s are fp32, correctly rounded;
+ *   - p = exp(score - M_t), M_t the running max of the 32-key walk after the
+ *     key's tile; the softmax normaliser sums the unquantised p, so the LSE
+ *     output is that of attn_paged_decode;
+ *   - with either operand quantised the decode always runs a 32-key skip
+ *     schedule (threshold 0 skips nothing): two passes over the splits with a
+ *     workspace of attn_paged_decode_qdq_workspace_size() bytes, or one
+ *     sequential split per (sequence, kv-head) with workspace NULL.
+ *
+ *   p_qdq, v_qdq        ATTN_QDQ_NONE or ATTN_QDQ_NVFP4
+ *   p_qdq_amax,
+ *   v_qdq_amax          the operand's calibrated absolute maximum, finite, in
+ *                       [2^-64, 2^64] when its format is NVFP4 (ignored
+ *                       otherwise); values above it saturate.  Probabilities
+ *                       never exceed 1, so 1 is the natural P amax.
+ *   other arguments     as attn_paged_decode_ex.  With both formats NONE
+ *                       the call is attn_paged_decode_ex.
+ * Errors as attn_paged_decode_ex, plus ATTN_E_QDQ.
+ */
+ATTN_API size_t attn_paged_decode_qdq_workspace_size(int batch, int h_q, int d, int max_pages_per_seq);
+ATTN_API int attn_paged_decode_qdq(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_bf16 *v_cache,
+                                   const int32_t *block_table, const int32_t *seq_lens, int batch,
+                                   int num_pages, int max_pages_per_seq, int page_size, int h_q, int h_kv,
+                                   int d, float skip_threshold, float scale, int p_qdq, float p_qdq_amax,
+                                   int v_qdq, float v_qdq_amax, uint32_t *skip_mask,
+                                   unsigned long long *skip_counts, attn_bf16 *out, float *lse,
+                                   void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * attn_paged_decode_static -- attn_paged_decode for callers that cannot

@@ -105,3 +105,25 @@ def host_bits(t):
 
 def dev_i32(a, device="cuda"):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+
+def assert_close_bf16_bound(gpu, ref, bound, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+    """assert_close_bf16 with a per-element allowance ``bound`` (>= 0) for
+    elements whose reference rests on a rounding decision the two sides may
+    take differently (a quantised code next to its rounding midpoint): such an
+    element may differ by max_abs + bound; the mean over elements without an
+    allowance stays under mean_abs.  Returns (max error, mean error, number
+    of elements with an allowance)."""
+    g = to_f64(gpu)
+    r = oracle.round_f64_to_bf16(np.asarray(ref, dtype=np.float64))
+    b = np.asarray(bound, dtype=np.float64)
+    mask = ~np.isnan(r)
+    assert mask.any(), "nothing to compare"
+    assert np.all(np.isfinite(g[mask])), "non-finite GPU output"
+    err = np.abs(g - r)
+    bad = mask & (err > max_abs + b)
+    assert not bad.any(), f"max-abs {err[bad].max():.3e} over {max_abs} + allowance at {np.argwhere(bad)[:3].tolist()}"
+    strict = mask & (b == 0)
+    if strict.any():
+        assert err[strict].mean() <= mean_abs, f"mean-abs {err[strict].mean():.3e} > {mean_abs}"
+    return float(err[mask].max()), float(err[strict].mean()) if strict.any() else 0.0, int((mask & (b > 0)).sum())

@@ -258,3 +258,35 @@ def test_static_decode_too_large_after_argument_checks(A):
     # a bad argument is reported as such even when the shape is too large
     assert static_decode(A, batch=3025, hq=1, hkv=1, d=96) == -4
     assert static_decode(A, batch=3025, hq=1, hkv=1, q=None) == -1
+
+
+def decode_qdq(A, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, batch=2, pages=4, maxp=2, ps=16, hq=8, hkv=2, d=128,
+             thr=0.0, scale=0.1, pf=1, pa=1.0, vf=1, va=1.0, mask=None, counts=None, out=FAKE, lse=None, ws=FAKE,
+             wsb=1 << 30, stream=None)
+    a.update(kw)
+    return A.lib.attn_paged_decode_qdq(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["batch"], a["pages"],
+                                       a["maxp"], a["ps"], a["hq"], a["hkv"], a["d"], a["thr"], a["scale"], a["pf"],
+                                       a["pa"], a["vf"], a["va"], a["mask"], a["counts"], a["out"], a["lse"], a["ws"],
+                                       a["wsb"], a["stream"])
+
+
+def test_decode_qdq_argument_errors(A):
+    assert decode_qdq(A, pf=2) == -14
+    assert decode_qdq(A, vf=-1) == -14
+    for bad in (0.0, -1.0, float("nan"), float("inf"), 2.0 ** 70, 2.0 ** -70):
+        assert decode_qdq(A, pa=bad) == -14
+        assert decode_qdq(A, va=bad) == -14
+    # an unused amax is not checked
+    assert decode_qdq(A, pf=0, pa=float("nan"), wsb=100) == -9
+    # the decode's own checks come first
+    assert decode_qdq(A, hq=7) == -3
+    assert decode_qdq(A, d=96) == -4
+    assert decode_qdq(A, thr=1.5) == -5
+    # with QDQ on, a workspace selects the two-pass skip schedule at any threshold
+    need = A.lib.attn_paged_decode_qdq_workspace_size(2, 8, 128, 2)
+    assert need == A.lib.attn_paged_decode_workspace_size_ex(2, 8, 128, 2, 0.5)
+    assert need > A.lib.attn_paged_decode_workspace_size(2, 8, 128)
+    assert decode_qdq(A, wsb=need - 1) == -9
+    assert decode_qdq(A, ws=FAKE + 4) == -2
+    assert A.lib.attn_status_string(-14) == b"ATTN_E_QDQ"
