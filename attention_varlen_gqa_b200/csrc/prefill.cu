@@ -834,6 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mref = (m_used == -INFINITY) ? 0.f : m_used;
         float um[4];                                // raw maxima of the four 32-key sub-tiles
         max_sub4(sr, um);
+        uint32_t wv = 0;                            // sub-tiles every row of this warp votes to skip
         if constexpr (SKIP) {
           // vote per 32-key sub-tile: exp(sub-tile max - running max) <
           // threshold for every row of the warp
@@ -845,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_true = fmaxf(m_true, t2);
             my_votes |= uint32_t(vote) << u;
           }
-          const uint32_t wv = __reduce_and_sync(0xffffffffu, my_votes);
+          wv = __reduce_and_sync(0xffffffffu, my_votes);
           if (lane == 0) {
             votes[(t * 3 + tile_c % 3) * 4 + quad] = wv;
             mbar_arrive(&votes_ready[2 * t + (tile_c & 1)]);
@@ -864,13 +865,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t skip = 0;                          // sub-tiles every row of the warpgroup skips
         if constexpr (SKIP) {
           // the four warps' votes (a warp is at most one tile ahead of the
-          // others: the next S needs every warp's P of this one)
-          if (!__all_sync(0xffffffffu, wait_or_abort(&votes_ready[2 * t + (tile_c & 1)], (tile_c >> 1) & 1,
-                                                     abort_flag, p.err))) {
-            alive = false;
-            return false;
+          // others: the next S needs every warp's P of this one).  A sub-tile
+          // is skipped only if every warp's word has its bit: a warp whose own
+          // word is 0 knows that none is and does not wait for the others.
+          if (wv != 0) {
+            if (!__all_sync(0xffffffffu, wait_or_abort(&votes_ready[2 * t + (tile_c & 1)], (tile_c >> 1) & 1,
+                                                       abort_flag, p.err))) {
+              alive = false;
+              return false;
+            }
+            skip = and4_shared(votes + (t * 3 + tile_c % 3) * 4);
           }
-          skip = and4_shared(votes + (t * 3 + tile_c % 3) * 4);
 #pragma unroll
           for (int u = 0; u < 2; ++u)
             ps[u] = ((skip >> u) & 1u) ? 0.f : exp32_to_tmem(sr[u], sl2, mref, tS + 16 * u);
