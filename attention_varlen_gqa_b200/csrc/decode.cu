@@ -318,11 +318,12 @@ ATTN_DEVICE void warp_pv_qdq(float (&o_acc)[D / 16][NH][4], float (&m_w)[NH][2],
       const uint32_t sc = e4m3x2_as_f16x2(__fmul_rn(bf16_lo(bm), p.v_k), __fmul_rn(bf16_hi(bm), p.v_k));
       const float r_g = ratio_from_table(f16_lo(sc), v_tab), r_g8 = ratio_from_table(f16_hi(sc), v_tab);
       const uint32_t s_g = f16x2_bcast(sc, false), s_g8 = f16x2_bcast(sc, true);
+      const uint64_t r2_g = f2_pack(r_g, r_g), r2_g8 = f2_pack(r_g8, r_g8);
       uint32_t f[4];
-      f[0] = qdq_bf16_pair(a[0], r_g, s_g);
-      f[1] = qdq_bf16_pair(a[1], r_g8, s_g8);
-      f[2] = qdq_bf16_pair(a[2], r_g, s_g);
-      f[3] = qdq_bf16_pair(a[3], r_g8, s_g8);
+      f[0] = qdq_bf16_pair(a[0], r2_g, s_g);
+      f[1] = qdq_bf16_pair(a[1], r2_g8, s_g8);
+      f[2] = qdq_bf16_pair(a[2], r2_g, s_g);
+      f[3] = qdq_bf16_pair(a[3], r2_g8, s_g8);
 #pragma unroll
       for (int n = 0; n < NH; ++n) mma_f16_16816(o_acc[mt_][n], f, pb[n][0], pb[n][1]);
     } else {

@@ -98,9 +98,15 @@ ATTN_DEVICE uint32_t max_bf16x2(uint32_t a, uint32_t b) {
 }
 
 // The dequantised pair (times g) of a bf16x2 pair of one block: its E2M1
-// codes at ratio r, times the block scale (f16x2 with both halves s).
-ATTN_DEVICE uint32_t qdq_bf16_pair(uint32_t x, float r, uint32_t s2) {
-  return hmul2_u32(e2m1x2_as_f16x2(__fmul_rn(bf16_lo(x), r), __fmul_rn(bf16_hi(x), r)), s2);
+// codes at ratio r (r2 = the pair (r, r)), times the block scale (f16x2 with
+// both halves s).  The two products are one packed fp32 multiply, each lane
+// rounded to nearest as a scalar product would be.
+ATTN_DEVICE uint32_t qdq_bf16_pair(uint32_t x, uint64_t r2, uint32_t s2) {
+  uint64_t y;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(f2_pack(bf16_lo(x), bf16_hi(x))), "l"(r2));
+  float y0, y1;
+  f2_unpack(y, y0, y1);
+  return hmul2_u32(e2m1x2_as_f16x2(y0, y1), s2);
 }
 
 // m16n8k16 MMA with f16 operands (fp32 accumulate).

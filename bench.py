@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "smallseq", "skip", "smallseq_bwd",
-                                       "decode_skip", "varlen_bwd", "paged_prefill"],
+                                       "decode_skip", "decode_qdq", "varlen_bwd", "paged_prefill"],
                     default="all",
                     help="profiling aid: run a single operation (no JSON line)")
     ap.add_argument("--no-skip", action="store_true",
@@ -288,7 +288,7 @@ def main():
 
     # ---------------- inputs (device-resident) ----------------
     want = {"prefill", "decode", "smallseq"} if args.only == "all" else {args.only}
-    if args.only == "decode_skip":
+    if args.only in ("decode_skip", "decode_qdq"):
         want = {"decode"}
     ops = []
     if "prefill" in want:
@@ -335,13 +335,15 @@ def main():
             A.attn_smallseq_fwd(ss["q"], ss["k"], ss["v"], ss_cu, 16, out=ss_out, weights=ss_w)
         ops.append(("smallseq", do_smallseq))
 
-    if args.only == "decode_skip":
-        # the decode workload in skip mode (threshold 0.1), two passes over the splits
+    if args.only in ("decode_skip", "decode_qdq"):
+        # the decode workload in skip mode (threshold 0.1), two passes over the
+        # splits; decode_qdq adds NVFP4 quantise-dequantise of P and V (amax 1)
+        qkw = dict(p_qdq="nvfp4", p_qdq_amax=1.0, v_qdq="nvfp4", v_qdq_amax=1.0) if args.only == "decode_qdq" else {}
         dsk_ws = torch.empty(A.attn_paged_decode_workspace_size(dec_batch, 32, 128, dec["block_table"].shape[1], 0.1),
                              dtype=torch.uint8, device=dev)
         for _ in range(args.warmup + args.steps):
             A.attn_paged_decode(dec["q"], dec["k_cache"], dec["v_cache"], dec_bt, dec_sl, skip_threshold=0.1,
-                                out=dec_out, lse=dec_lse, workspace=dsk_ws)
+                                out=dec_out, lse=dec_lse, workspace=dsk_ws, **qkw)
         torch.cuda.synchronize()
         assert A.attn_get_last_device_error() == 0
         return

@@ -85,3 +85,87 @@ def test_reference_arm_prints_once_under_torchrun():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+# ---------------------------------------------------------------------------
+# one varlen batch sharded by whole sequences across ranks
+# ---------------------------------------------------------------------------
+
+def test_sequence_cost_counts_allowed_pairs():
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    from attention_varlen_gqa_b200 import shard
+    for s_q, s_k in ((1, 1), (5, 5), (7, 3), (3, 9), (0, 4), (4, 0), (128, 300)):
+        for causal in (True, False):
+            want = int(oracle.allowed_mask(s_q, s_k, causal).sum()) if s_q and s_k else 0
+            assert shard.sequence_cost(s_q, s_k, causal) == want
+
+
+def test_lpt_partition_properties():
+    sys.path.insert(0, ROOT)
+    from attention_varlen_gqa_b200 import shard
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for world in (1, 2, 3, 8):
+        costs = rng.integers(0, 10_000, 37).tolist()
+        parts = shard.lpt_partition(costs, world)
+        assert len(parts) == world
+        flat = sorted(i for p in parts for i in p)
+        assert flat == list(range(len(costs)))                       # each sequence exactly once
+        loads = [sum(costs[i] for i in p) for p in parts]
+        lower = max(sum(costs) / world, max(costs))
+        assert max(loads) <= (4 / 3) * lower + 1e-9                  # the list-scheduling bound
+        assert parts == shard.lpt_partition(costs, world)           # deterministic
+    assert shard.lpt_partition([5, 5, 5], 1) == [[0, 1, 2]]
+
+
+def _shard_worker(rank, world, port, out_path):
+    import datetime
+
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    import workloads as W
+    from attention_varlen_gqa_b200 import shard
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        lens_q = [70, 0, 129, 33, 200, 5, 64]
+        lens_k = [70, 16, 150, 33, 230, 5, 64]
+        data = W.varlen_prefill(lens_q, lens_k, h_q=4, h_kv=2, d=64, causal=True, seed=7)
+        parts = shard.shard_varlen(lens_q, lens_k, True, world)
+        mine = parts[rank]
+        rq, cq = shard.shard_rows(data["cu_seqlens_q"], mine)
+        rk, ck = shard.shard_rows(data["cu_seqlens_k"], mine)
+        out, lse, _ = oracle.varlen_attention(data["q"][rq], data["k"][rk], data["v"][rk], cq, ck, 4, 2, True,
+                                              data["scale"])
+        got = [None] * world
+        dist.all_gather_object(got, (mine, rq.tolist(), out, lse))
+        if rank == 0:
+            full_o = np.full((int(data["cu_seqlens_q"][-1]), 4, 64), np.nan)
+            full_l = np.full((int(data["cu_seqlens_q"][-1]), 4), np.nan)
+            for seqs, rows, o, l in got:
+                full_o[rows] = o
+                full_l[rows] = l
+            ref_o, ref_l, _ = oracle.varlen_attention(data["q"], data["k"], data["v"], data["cu_seqlens_q"],
+                                                      data["cu_seqlens_k"], 4, 2, True, data["scale"])
+            same = bool(np.array_equal(full_o, ref_o, equal_nan=True) and np.array_equal(full_l, ref_l))
+            with open(out_path, "w") as f:
+                json.dump({"same": same, "parts": parts}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_batch_equals_unsharded(tmp_path):
+    """Two gloo ranks each take their LPT share of one varlen batch (whole
+    sequences, heaviest first to the least-loaded rank), compute it on its own
+    (here with the fp64 oracle), and the gathered results equal the unsharded
+    computation exactly: the sequences are independent problems."""
+    out = tmp_path / "shard.json"
+    mp.start_processes(_shard_worker, args=(2, free_port(), str(out)), nprocs=2, join=True, start_method="spawn")
+    res = json.loads(out.read_text())
+    assert res["same"]
+    assert sorted(i for p in res["parts"] for i in p) == list(range(7))
+    assert all(len(p) > 0 for p in res["parts"])
