@@ -127,3 +127,13 @@ def assert_close_bf16_bound(gpu, ref, bound, max_abs=MAX_ABS, mean_abs=MEAN_ABS)
     if strict.any():
         assert err[strict].mean() <= mean_abs, f"mean-abs {err[strict].mean():.3e} > {mean_abs}"
     return float(err[mask].max()), float(err[strict].mean()) if strict.any() else 0.0, int((mask & (b > 0)).sum())
+
+
+# Largest errors seen per check, against their bounds: printed at the end of
+# the run (tests/conftest.py) so that a tolerance's headroom is visible.
+HEADROOM = {}
+
+
+def record_headroom(name, max_err, max_bound, mean_err, mean_bound):
+    old = HEADROOM.get(name, (0.0, max_bound, 0.0, mean_bound))
+    HEADROOM[name] = (max(old[0], max_err), max_bound, max(old[2], mean_err), mean_bound)

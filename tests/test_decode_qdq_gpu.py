@@ -221,3 +221,33 @@ def test_qdq_full_size_sampled(A, thr, schedule):
     data = W.skip_decode(seed=0, where="device")
     batches = [0, 13, 31]
     _check(A, data, thr, schedule, 1.0, 1.0, t=_dev(data), batches=batches, host=_sampled_host(data, batches))
+
+
+@pytest.mark.parametrize("schedule", ["split", "sequential"])
+def test_qdq_bad_block_table_entry(A, schedule):
+    """A block-table entry outside the pool sets ATTN_DEVERR_BLOCK_TABLE and
+    zeroes that sequence's output, with QDQ on as without; the other
+    sequence still matches the oracle."""
+    data = W.paged_decode([40, 50], h_q=4, h_kv=2, d=128, seed=3)
+    bt = data["block_table"].copy()
+    bt[1, 2] = data["num_pages"] + 5
+    data["block_table"] = bt
+    t = _dev(data)
+    for thr in (0.0, 0.1):
+        out, lse, _, _, _ = _run(A, data, t, thr, schedule, 1.0, 2.0)
+        assert A.attn_get_last_device_error() & 4
+        assert torch.all(out[1] == 0)
+        assert torch.all(torch.isneginf(lse[1]))
+        ro, rl, _, flip = N.paged_decode_qdq(data["q"], data["k_cache"], data["v_cache"], bt, data["seq_lens"], 4,
+                                             2, data["scale"], threshold=thr, p_amax=1.0, v_amax=2.0, batches=[0])
+        assert_close_bf16_bound(out[0], ro[0], flip[0])
+
+
+def test_qdq_seq_len_beyond_table(A):
+    data = W.paged_decode([40, 50], h_q=4, h_kv=2, d=64, seed=4)
+    sl = data["seq_lens"].copy()
+    sl[0] = data["block_table"].shape[1] * 16 + 1
+    data["seq_lens"] = sl
+    out, lse, _, _, _ = _run(A, data, _dev(data), 0.0, "split", 1.0, None)
+    assert A.attn_get_last_device_error() & 2
+    assert torch.all(out[0] == 0)
