@@ -34,6 +34,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -88,9 +89,9 @@ struct Smem {
   static constexpr int kStageBytes = BM * 64 * 2;
   static constexpr int kStage = kV + kStages * kTile;
   static constexpr int kBar = kStage + kNQ * kStageBytes;
-  // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], o_free[NQ],
-  // p_half[NQ], sched_full[SD], sched_empty[SD], votes_ready[NQ][2]
-  static constexpr int kNumBars = 2 + 3 * kStages + 5 * kNQ + 2 * kSchedDepth + 2 * kNQ;
+  // q_full, q_empty, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[NQ], p_full[NQ], o_done[NQ],
+  // o_free[NQ], p_half[NQ], sched_full[SD], sched_empty[SD], votes_ready[NQ][2]
+  static constexpr int kNumBars = 2 + 4 * kStages + 5 * kNQ + 2 * kSchedDepth + 2 * kNQ;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static_assert(kMisc % 16 == 0, "the vote words are read as 16-byte vectors");
   static constexpr int kUsed = kMisc + 128;
@@ -365,7 +366,7 @@ ATTN_DEVICE float exp32_to_tmem(const uint32_t (&a)[32], float sl2, float mref, 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int D, bool SKIP>
+template <int D, bool SKIP, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
@@ -378,8 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *q_empty = q_full + 1;
   uint64_t *k_full = q_empty + 1;
   uint64_t *v_full = k_full + kStages;
-  uint64_t *kv_empty = v_full + kStages;
-  uint64_t *s_full = kv_empty + kStages;
+  uint64_t *k_empty = v_full + kStages;         // [S] both tiles' S of the slot's K tile are done
+  uint64_t *v_empty = k_empty + kStages;        // [S] both tiles' P.V of the slot's V tile are done
+  uint64_t *s_full = v_empty + kStages;
   uint64_t *p_full = s_full + kNQ;
   uint64_t *o_done = p_full + kNQ;
   uint64_t *o_free = o_done + kNQ;
@@ -424,7 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int t = 0; t < kNQ; ++t) {
       mbar_init(&s_full[t], 1);
@@ -465,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const uint64_t keep = policy_evict_last();     // K/V tiles are re-read by other q-heads
       uint32_t kv_c = 0, q_c = 0;
+      uint32_t k_issued = 0, v_issued = 0;    // K / V tiles whose copies were issued
       bool ok = true;
       auto wait_all_p = [&](uint64_t *bar, uint32_t parity) {
         return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, p.err));
@@ -496,33 +500,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const int hk = it.hq[0] / p.group;
-        const int32_t *bt = p.paged ? p.block_table + (size_t)it.b * p.max_pages : nullptr;
+        const int32_t *bt = PAGED ? p.block_table + (size_t)it.b * p.max_pages : nullptr;
         // a paged tile's block-table entries are read one tile ahead, so that
-        // their latency is not added to the copies' once the stage frees up
+        // their latency is not added to the copies' once a slot frees up
         auto page_raw = [&](int j) -> int {
           const int tok = j * BN + lane * kPageSize;
-          return (p.paged && lane < BN / kPageSize && tok < sq.s_k) ? __ldg(bt + tok / kPageSize) : 0;
+          return (PAGED && lane < BN / kPageSize && tok < sq.s_k) ? __ldg(bt + tok / kPageSize) : 0;
         };
-        int raw_next = page_raw(0);
-        for (int j = 0; j < nmax; ++j, ++kv_c) {
-          const int s = kv_c % kStages;
-          const int raw = raw_next;
-          if (j + 1 < nmax) raw_next = page_raw(j + 1);
-          if (kv_c >= kStages && !(ok = wait_all_p(&kv_empty[s], ((kv_c / kStages) - 1) & 1))) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&k_full[s], BN * D * 2);
-            mbar_arrive_expect_tx(&v_full[s], BN * D * 2);
-          }
+        // K or V tile j of the item (global tile count c) into its ring slot,
+        // once the slot's previous tile is no longer read
+        auto load = [&](bool is_k, int j, uint32_t c, int raw) -> bool {
+          const int s = c % kStages;
+          uint64_t *full = is_k ? k_full : v_full;
+          if (c >= kStages && !wait_all_p(is_k ? &k_empty[s] : &v_empty[s], ((c / kStages) - 1) & 1))
+            return false;
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], BN * D * 2);
           __syncwarp();
-          if (!p.paged) {
-            if (lane == 0) {
+          const CUtensorMap *map = is_k ? &kmap : &vmap;
+          uint8_t *slot = sm + (is_k ? L::kK : L::kV) + s * L::kTile;
+          if constexpr (!PAGED) {
+            if (lane == 0)
               for (int h = 0; h < D / 64; ++h)
-                tma_load_3d_hint(sm + L::kK + s * L::kTile + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
-                                 sq.k0 + j * BN, keep);
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_3d_hint(sm + L::kV + s * L::kTile + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
-                                 sq.k0 + j * BN, keep);
-            }
+                tma_load_3d_hint(slot + h * BN * 128, map, &full[s], h * 64, hk, sq.k0 + j * BN, keep);
           } else if (lane < BN / kPageSize) {
             // one 16-token page per box; a page past the sequence (or a bad
             // block-table entry, reported) is read at a row beyond the cache,
@@ -532,29 +531,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tok < sq.s_k) {
               page = raw;
               if (page < 0 || page >= p.num_pages) {
-                raise_error(p.err, ATTN_DEVERR_BLOCK_TABLE);
+                if (is_k) raise_error(p.err, ATTN_DEVERR_BLOCK_TABLE);
                 page = p.num_pages;
               }
             }
-            const uint32_t off = s * L::kTile + lane * kPageSize * 128;
-            for (int h = 0; h < D / 64; ++h) {
-              tma_load_3d_hint(sm + L::kK + off + h * BN * 128, &kmap, &k_full[s], h * 64, hk,
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d_hint(slot + lane * kPageSize * 128 + h * BN * 128, map, &full[s], h * 64, hk,
                                page * kPageSize, keep);
-              tma_load_3d_hint(sm + L::kV + off + h * BN * 128, &vmap, &v_full[s], h * 64, hk,
-                               page * kPageSize, keep);
-            }
           }
           __syncwarp();
+          return true;
+        };
+        // K runs one tile ahead of V: a K slot frees when both query tiles'
+        // S of its tile are done, a V slot only when their P.V are, so the
+        // next K tile (which the next S waits for) is fetched a tile earlier
+        int raw0 = page_raw(0), raw1 = nmax > 1 ? page_raw(1) : 0;
+        if (!(ok = load(true, 0, kv_c, raw0))) break;
+        k_issued = kv_c + 1;
+        for (int j = 0; j < nmax; ++j) {
+          const int raw2 = j + 2 < nmax ? page_raw(j + 2) : 0;
+          if (j + 1 < nmax) {
+            if (!(ok = load(true, j + 1, kv_c + j + 1, raw1))) break;
+            k_issued = kv_c + j + 2;
+          }
+          if (!(ok = load(false, j, kv_c + j, raw0))) break;
+          v_issued = kv_c + j + 1;
+          raw0 = raw1;
+          raw1 = raw2;
         }
+        if (!ok) break;
+        kv_c += nmax;
         ++q_c;
       }
       if (!ok && lane == 0) {
         // let copies still in flight land before the CTA's shared memory is released
         if (q_c > 0) drain(q_full, (q_c - 1) & 1);
-        for (uint32_t x = kv_c > kStages ? kv_c - kStages : 0; x < kv_c; ++x) {
+        for (uint32_t x = k_issued > kStages ? k_issued - kStages : 0; x < k_issued; ++x)
           drain(&k_full[x % kStages], (x / kStages) & 1);
+        for (uint32_t x = v_issued > kStages ? v_issued - kStages : 0; x < v_issued; ++x)
           drain(&v_full[x % kStages], (x / kStages) & 1);
-        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -619,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int t = 0; t < kNQ; ++t)
         if (g[t].n > 0) issue_s(t, kv_c % kStages);
+      commit(&k_empty[kv_c % kStages]);
       uint32_t pv_started[kNQ] = {0, 0};
       for (int j = 0; ok && j < nmax; ++j) {
         const uint32_t c = kv_c + j, st = c % kStages;
@@ -641,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
             tc_fence_after();
             v_ready = true;
-            if (p.paged && j == (sq.s_k - 1) / BN && (sq.s_k % kPageSize) != 0) {
+            if (PAGED && j == (sq.s_k - 1) / BN && (sq.s_k % kPageSize) != 0) {
               // the sequence's last page holds slots past its end (whatever the
               // cache has there); their p is 0, but 0 * NaN is not, so the V
               // rows are zeroed before the P.V MMAs read them
@@ -693,7 +709,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_s(t, (c + 1) % kStages);
           }
         }
-        if (ok) commit(&kv_empty[st]);
+        if (ok) {
+          // this tile's V, and the next tile's K once both S were issued above
+          commit(&v_empty[st]);
+          if (j + 1 < nmax) commit(&k_empty[(c + 1) % kStages]);
+        }
       }
       if (!ok) break;
       commit(q_empty);
@@ -1065,11 +1085,11 @@ int num_sms() {
   return n;
 }
 
-template <int D, bool SKIP>
+template <int D, bool SKIP, bool PAGED>
 cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
                      const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t stream) {
   const int smem = Smem<D>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, SKIP>,
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, SKIP, PAGED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long items = (p.group % 2 == 0) ? (long long)p.batch * p.qb_max * (p.h_q / 2)
@@ -1080,7 +1100,7 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &qmap, const CUte
   PrefillParams q = p;
   q.work_tag = next_tag.fetch_add(1u) % 0xffffffffu + 1u;
   q.work_slot = (int)(q.work_tag % kWorkSlots);
-  prefill_kernel<D, SKIP><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, omap, q);
+  prefill_kernel<D, SKIP, PAGED><<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, omap, q);
   return cudaGetLastError();
 }
 
@@ -1090,11 +1110,17 @@ cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap, cons
                            const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t stream) {
   if (p.batch == 0 || p.qb_max == 0) return cudaSuccess;
   const bool skip = p.thr_log2 > -INFINITY;
+  // one instantiation per (head dim, skip, paged): each keeps only its own
+  // load and softmax code
+  auto go = [&](auto d, auto sk) {
+    return p.paged ? launch_t<decltype(d)::value, decltype(sk)::value, true>(p, qmap, kmap, vmap, omap, stream)
+                   : launch_t<decltype(d)::value, decltype(sk)::value, false>(p, qmap, kmap, vmap, omap, stream);
+  };
+  using T = std::true_type;
+  using F = std::false_type;
   if (p.d == 128)
-    return skip ? launch_t<128, true>(p, qmap, kmap, vmap, omap, stream)
-                : launch_t<128, false>(p, qmap, kmap, vmap, omap, stream);
-  return skip ? launch_t<64, true>(p, qmap, kmap, vmap, omap, stream)
-              : launch_t<64, false>(p, qmap, kmap, vmap, omap, stream);
+    return skip ? go(std::integral_constant<int, 128>{}, T{}) : go(std::integral_constant<int, 128>{}, F{});
+  return skip ? go(std::integral_constant<int, 64>{}, T{}) : go(std::integral_constant<int, 64>{}, F{});
 }
 
 }  // namespace attn
