@@ -653,7 +653,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // their row sums; sub-tiles past the keys vote skip too).
           uint32_t skip_bits = 0;
           if constexpr (SKIP) skip_bits = and4_shared(votes + (t * 3 + vslot[t]) * 4);
-          if (!v_ready) {
+          // With both sub-tiles of keys [64, 128) skipped the softmax warps
+          // write nothing to this tile's TMEM after their first hand-off (S
+          // is in their registers by then), so the next S is issued without
+          // waiting for the second; with all four skipped, no P.V reads V.
+          const bool hi_skip = SKIP && (skip_bits & 0xcu) == 0xcu;
+          const bool all_skip = SKIP && (skip_bits & 0xfu) == 0xfu;
+          if (!v_ready && !all_skip) {
             if (!(ok = wait_all(&v_full[st], (c / kStages) & 1))) continue;
             tc_fence_after();
             v_ready = true;
@@ -685,14 +691,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           __syncwarp();
-          if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) continue;
-          tc_fence_after();
-          if (leader) {
+          if (!hi_skip) {
+            // (a skipped wait is safe: this p_full phase completes before the
+            // next p_half one, which the next step waits for first)
+            if (!(ok = wait_all(&p_full[t], tile_c[t] & 1))) continue;
+            tc_fence_after();
+            if (leader) {
 #pragma unroll
-            for (int kk = BN / 32; kk < BN / 16; ++kk) {
-              if ((skip_bits >> (kk / 2)) & 1u) continue;
-              mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, acc);
-              acc = 1u;
+              for (int kk = BN / 32; kk < BN / 16; ++kk) {
+                if ((skip_bits >> (kk / 2)) & 1u) continue;
+                mma_ts(d, a + kk * 8, v0 + ((kk * 16 * 128) >> 4), idPV, acc);
+                acc = 1u;
+              }
             }
           }
           pv_started[t] = __shfl_sync(0xffffffffu, acc, leader_lane);
@@ -709,6 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_s(t, (c + 1) % kStages);
           }
         }
+        // the V slot is released only after its copy has landed, read or not
+        if (ok && !v_ready) ok = wait_all(&v_full[st], (c / kStages) & 1);
         if (ok) {
           // this tile's V, and the next tile's K once both S were issued above
           commit(&v_empty[st]);
@@ -722,10 +734,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       kv_c += nmax;
       ++q_c;
     }
-    // every MMA must be complete before the TMEM is released
+    // every MMA must be complete before the TMEM is released, and every
+    // commit's arrival must have landed before the shared memory is
+    if (leader) {
 #pragma unroll
-    for (int t = 0; t < kNQ; ++t)
-      if (tile_c[t] > 0) drain(&o_done[t], (tile_c[t] - 1) & 1);
+      for (int t = 0; t < kNQ; ++t)
+        if (tile_c[t] > 0) drain(&o_done[t], (tile_c[t] - 1) & 1);
+      if (kv_c > 0) {
+        drain(&k_empty[(kv_c - 1) % kStages], ((kv_c - 1) / kStages) & 1);
+        drain(&v_empty[(kv_c - 1) % kStages], ((kv_c - 1) / kStages) & 1);
+      }
+      if (q_c > 0) drain(q_empty, (q_c - 1) & 1);
+    }
+    __syncwarp();
   } else if (warp == kSchedWarp) {
     // =============== work claims ===============
     if (ranked(p)) {
