@@ -762,9 +762,8 @@ struct SplitRange {
 // that publishes them, so loads it issues share their round trip.
 template <typename Extra>
 ATTN_DEVICE SplitRange split_range(const DecodeParams &p, int b, int split, int32_t *bt_s, int bt_cap,
-                                   Extra extra) {
+                                   Extra extra, int L) {
   SplitRange r;
-  int L = __ldg(p.seq_lens + b);
   const bool bad_len = (L < 0) | (L > p.max_pages * kPageSize);
   if (bad_len) L = 0;
   const int n_chunks_all = (L + kChunk - 1) / kChunk;
@@ -806,7 +805,7 @@ __global__ void __launch_bounds__(kThreads) decode_scores_kernel(const __grid_co
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int G = p.group;
   const SplitRange r = split_range(p, b, split, reinterpret_cast<int32_t *>(base + Lay::kBt), Lay::kBtCap,
-                                   [](int, int, int) {});
+                                   [](int, int, int) {}, __ldg(p.seq_lens + b));
   const int n = r.c1 - r.c0;
   const size_t seq = (size_t)b * p.h_kv + hk;
   float *S = p.ws_s + seq * (size_t)p.s_stride * G;          // [token][G]
@@ -877,6 +876,19 @@ __global__ void __launch_bounds__(kThreads) decode_scores_kernel(const __grid_co
   }
 }
 
+// ORs bits [u0, u1) of a bit mask in global memory, a word at a time.
+ATTN_DEVICE void or_bit_range(uint32_t *mask, long long u0, long long u1) {
+  while (u0 < u1) {
+    const long long w = u0 >> 5;
+    const int lo = (int)(u0 & 31);
+    const long long span = u1 - (w << 5);
+    const int hi = span < 32 ? (int)span : 32;
+    const uint32_t bits = (hi == 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~((1u << lo) - 1u);
+    atomicOr(mask + w, bits);
+    u0 = (w + 1) << 5;
+  }
+}
+
 template <int D, int NH, bool QDQ>
 __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_constant__ CUtensorMap vmap,
                                                                   DecodeParams p) {
@@ -898,12 +910,12 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
 
   // with the block-table entries, in the same round trip: the split's tile
   // maxima and the earlier splits' maxima, to shared memory
-  float *sm_s = reinterpret_cast<float *>(base + Lay::kX);   // [split][G], earlier splits
+  float *sm_s = reinterpret_cast<float *>(base + Lay::kX);   // [split][G], this and earlier splits
   const SplitRange r = split_range(
       p, b, split, reinterpret_cast<int32_t *>(base + Lay::kBt), Lay::kBtCap, [&](int L, int c0, int c1) {
         const int nt = max(0, min((L + kSkipTile - 1) / kSkipTile, 2 * c1) - 2 * c0);
         const int ntm = (2 * (c1 - c0) * G <= kTmaxCap) ? nt * G : 0;
-        const int nsm = split * G;
+        const int nsm = (split + 1) * G;   // (with this split's own)
         const float *tsrc = tmax + (size_t)2 * c0 * G;
         const float *ssrc = p.ws_smax + seq * kDecodeSplits * G;
         const float a = tid < ntm ? tsrc[tid] : 0.f;
@@ -912,7 +924,8 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
         if (tid < nsm) sm_s[tid] = c;
         for (int x = tid + kThreads; x < ntm; x += kThreads) tm_s[x] = tsrc[x];
         for (int x = tid + kThreads; x < nsm; x += kThreads) sm_s[x] = ssrc[x];
-      });
+      },
+      __ldg(p.seq_lens + b));
   const int n = r.c1 - r.c0;
   const bool tm_local = 2 * n * G <= kTmaxCap;
 
@@ -943,9 +956,37 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
     }
     float m_run = -INFINITY;   // head lane's running max entering the next tile
     unsigned long long n_vis = 0, n_skip = 0;
-    if (ln.w == 0 && head)
-      for (int s2 = 0; s2 < split; ++s2) m_run = fmaxf(m_run, sm_s[s2 * G + ln.lane]);
-    __syncthreads();   // barrier init
+    // A split whose maximum (per head, from the first pass) is below the
+    // threshold relative to the earlier splits' maximum has every tile
+    // skipped: the running max entering any of its tiles is at least that,
+    // and no tile max exceeds the split's.  It is settled here, with no ring:
+    // its tiles are counted and marked skipped, and it leaves an empty partial.
+    bool all_skipped = true;
+    if (ln.w == 0) {
+      for (int h = 0; h < G; ++h) {
+        const float mp = warp_max(ln.lane < split ? sm_s[ln.lane * G + h] : -INFINITY);
+        if (ln.lane == h) m_run = mp;   // the earlier splits' maximum
+        const float mine = sm_s[split * G + h];
+        all_skipped = all_skipped && (mine == -INFINITY || mine - mp < p.thr_log2);
+      }
+    }
+    if (__syncthreads_and(all_skipped)) {   // (also publishes the barrier init)
+      const int t0 = 2 * r.c0, t1 = min((r.L + kSkipTile - 1) / kSkipTile, 2 * r.c1);
+      if (tid == 0 && t1 > t0) {
+        if (p.skip_counts) {
+          atomicAdd(p.skip_counts + 0, (unsigned long long)(t1 - t0));
+          atomicAdd(p.skip_counts + 1, (unsigned long long)(t1 - t0));
+        }
+        if (p.skip_mask)
+          or_bit_range(p.skip_mask, (long long)seq * p.kt_max + t0, (long long)seq * p.kt_max + t1);
+      }
+      if (tid < G) {
+        const size_t row = ((size_t)b * p.h_q + (size_t)hk * G + tid) * kDecodeSplits + split;
+        p.ws_ml[row * 2 + 0] = -INFINITY;
+        p.ws_ml[row * 2 + 1] = 0.f;
+      }
+      return;
+    }
     // decide() leaves the head lane's running max after each of the chunk's
     // tiles in dm[] (the reference max of the quantised P)
     float dm[2] = {-INFINITY, -INFINITY};
