@@ -496,6 +496,7 @@ int paged_decode_impl(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_b
     }
     p.qdq_out = inv;
   }
+  size_t one_pass_clear = 0;   // bytes to zero at ws_s before a one-pass launch
   if (two_pass && batch > 0) {
     const SkipWorkspace w = skip_workspace(batch, h_q, d, max_pages_per_seq);
     char *base = static_cast<char *>(workspace);
@@ -505,6 +506,21 @@ int paged_decode_impl(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_b
     p.ws_tmax = reinterpret_cast<float *>(base + w.tmax);
     p.ws_smax = reinterpret_cast<float *>(base + w.smax);
     p.s_stride = w.s_stride;
+    // Without quantisation, and when a split's scores fit in shared memory,
+    // one pass replaces the two: each split's CTA keeps its scores on chip and
+    // waits for the earlier splits' maxima.  Its ticket counter and published
+    // maxima take the start of the scores area, zeroed before the launch.
+    const long long n128 = ((long long)max_pages_per_seq * kPageSize + kDecodeSplitTile - 1) / kDecodeSplitTile;
+    const int split_keys = (int)((n128 + kDecodeSplits - 1) / kDecodeSplits) * kDecodeSplitTile;
+    const size_t pub_bytes = (size_t)batch * h_q * kDecodeSplits * sizeof(unsigned long long);
+    if (!quant && decode_one_pass_smem(d, h_q / h_kv, split_keys) != 0 &&
+        256 + pub_bytes <= w.tmax - w.s) {
+      p.sequential = 3;
+      p.split_keys = split_keys;
+      p.ws_ticket = reinterpret_cast<unsigned int *>(base + w.s);
+      p.ws_pub = reinterpret_cast<unsigned long long *>(base + w.s + 256);
+      one_pass_clear = 256 + pub_bytes;
+    }
   }
   p.err = err;
 
@@ -516,6 +532,7 @@ int paged_decode_impl(const attn_bf16 *q, const attn_bf16 *k_cache, const attn_b
   if (skip_counts && cudaMemsetAsync(skip_counts, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
     return ATTN_E_CUDA;
   if (batch == 0) return ATTN_OK;
+  if (one_pass_clear && cudaMemsetAsync(p.ws_s, 0, one_pass_clear, st) != cudaSuccess) return ATTN_E_CUDA;
 
   CUtensorMap kmap, vmap;
   const long long slots = (long long)num_pages * page_size;

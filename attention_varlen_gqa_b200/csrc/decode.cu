@@ -1160,6 +1160,346 @@ __global__ void __launch_bounds__(kThreads) decode_skip_pv_kernel(const __grid_c
                          ln);
 }
 
+// ---------------------------------------------------------------------------
+// Skip mode in one pass over the split schedule
+// ---------------------------------------------------------------------------
+// One CTA per (split, kv-head, sequence) computes its split's scores into
+// shared memory (K chunks through the ring), publishes the split's maximum
+// per head, takes the earlier splits' maxima from the CTAs that computed them,
+// and then walks its 32-key tiles with the running max they give, copying the
+// V chunks of kept tiles through the same ring.  The decisions are the two
+// passes' (and the sequential walk's); the scores never leave the SM.  CTAs
+// take their split from a ticket counter in start order, splits innermost,
+// so every split a CTA waits for belongs to a CTA that started before it.
+// (Parking the scores in tensor memory instead, with a third ring stage in
+// the shared memory that frees, measured slower.)
+constexpr int kOneStages = 2;
+constexpr int kOneBtCap = 256;
+
+struct OnePassLayout {
+  size_t ring, sc, tm, qx, bt, keep, bar, total;
+  __host__ __device__ OnePassLayout(int d, int group, int split_keys) {
+    const size_t slot = (size_t)kChunk * d * 2;
+    ring = 0;
+    sc = ring + kOneStages * slot;                                   // [split_keys][G] scores
+    tm = sc + (((size_t)split_keys * group * 4 + 15) & ~size_t(15)); // [split_keys / 32][G] tile maxima
+    qx = tm + (((size_t)(split_keys / kSkipTile) * group * 4 + 15) & ~size_t(15));   // [2][warp][16]
+    bt = qx + 2 * kWarps * 16 * 4;                                   // block-table entries
+    keep = bt + kOneBtCap * 4;                                       // [stage] bits, [stage] chunk
+    bar = keep + 2 * kOneStages * 4;                                 // [stage] mbarriers
+    total = bar + kOneStages * 8;
+  }
+};
+
+template <int D, int NH>
+__global__ void __launch_bounds__(kThreads) decode_one_pass_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                   const __grid_constant__ CUtensorMap vmap,
+                                                                   DecodeParams p) {
+  constexpr int kSlot = kChunk * D * 2;
+  constexpr int S = kOneStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(base);
+  const int G = p.group;
+  const OnePassLayout lay(D, G, p.split_keys);
+  float *sc_s = reinterpret_cast<float *>(base + lay.sc);
+  float *tm_s = reinterpret_cast<float *>(base + lay.tm);
+  float *qx = reinterpret_cast<float *>(base + lay.qx);
+  uint32_t *keep_s = reinterpret_cast<uint32_t *>(base + lay.keep);
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + lay.bar);
+  const int tid = threadIdx.x;
+  const Lane ln(tid);
+  __shared__ int ticket;
+  if (tid == 0) ticket = (int)atomicAdd(p.ws_ticket, 1u);
+  __syncthreads();
+  const int split = ticket % kDecodeSplits;
+  const int hk = (ticket / kDecodeSplits) % p.h_kv;
+  const int b = ticket / (kDecodeSplits * p.h_kv);
+  const size_t seq = (size_t)b * p.h_kv + hk;
+  unsigned long long *pub = p.ws_pub + seq * kDecodeSplits * G;   // [split][G]
+
+  const SplitRange r = split_range(p, b, split, reinterpret_cast<int32_t *>(base + lay.bt), kOneBtCap,
+                                   [](int, int, int) {}, __ldg(p.seq_lens + b));
+  const int n = r.c1 - r.c0;
+  bool failed = false;
+  float smax = -INFINITY;   // thread (tt, h) = tid (tt * G + h): head h's max over tiles tt of each chunk
+
+  // ---- first half: the split's scores and tile maxima (K chunks) ----
+  if (!r.dead && n > 0) {
+    if (tid == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      for (int st = 0; st < S; ++st) mbar_init(&full[st], 1);
+      fence_barrier_init();
+    }
+    uint32_t qb[NH][D / 16][2];
+    load_q_frags<D, NH>(qb, p.q + ((size_t)b * p.h_q + (size_t)hk * G) * D, G, ln);
+    __syncthreads();
+    int issued = 0;
+    auto issue_k = [&](int c) {
+      const int st = c % S;
+      issue_pages<D>(&kmap, base + st * kSlot, &full[st], r.pages, (r.c0 + c) * kChunk, r.L, hk, 0, 4, true);
+    };
+    if (tid == 0)
+      for (; issued < min(n, S); ++issued) issue_k(issued);
+    for (int i = 0; i < n; ++i) {
+      const int st = i % S;
+      const bool ok = mbar_wait(&full[st], (i / S) & 1, p.err);
+      if (ok) {
+        const int tok_base = (r.c0 + i) * kChunk + ln.w * 16;
+        float sc[NH][4], qm[NH][2];
+        warp_scores<D, NH>(sc, qm, sbase + st * kSlot, qb, tok_base, r.L, G, p.scale_log2, ln);
+#pragma unroll
+        for (int nn = 0; nn < NH; ++nn) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tl = ln.w * 16 + ln.g + 8 * (e >> 1);
+            const int h = 8 * nn + ln.cq + (e & 1);
+            if (h < G) sc_s[((size_t)i * kChunk + tl) * G + h] = sc[nn][e];
+          }
+          if (ln.g == 0) {
+            qx[((i & 1) * kWarps + ln.w) * 16 + 8 * nn + ln.cq] = qm[nn][0];
+            qx[((i & 1) * kWarps + ln.w) * 16 + 8 * nn + ln.cq + 1] = qm[nn][1];
+          }
+        }
+      }
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      // every warp is done with stage st; chunk i's 16-key maxima are visible
+      if (tid == 0 && issued < n) issue_k(issued++);
+      if (tid < 2 * G) {
+        const int tt = tid / G, h = tid % G;
+        const float *x = qx + (i & 1) * kWarps * 16;
+        const float tmv = fmaxf(x[(2 * tt) * 16 + h], x[(2 * tt + 1) * 16 + h]);
+        tm_s[(2 * i + tt) * G + h] = tmv;
+        smax = fmaxf(smax, tmv);
+      }
+    }
+    if (failed && tid == 0)
+      for (int x = issued - min(S, issued); x < issued; ++x) mbar_wait(&full[x % S], (x / S) & 1, nullptr);
+  }
+
+  // ---- publish this split's maximum per head (every split, so that none waits in vain) ----
+  float own = -INFINITY;   // warp 0, lane h < G: head h's maximum over this split
+  if (tid < 32) {
+    const float other = __shfl_sync(0xffffffffu, smax, (tid + G) & 31);
+    own = fmaxf(smax, other);
+    if (tid < G) {
+      const unsigned long long w = (1ull << 32) | __float_as_uint(own);
+      asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(pub + split * G + tid), "l"(w) : "memory");
+    }
+  }
+
+  float o_acc[D / 16][NH][4];
+  float m_w[NH][2], l_w[NH][2];
+#pragma unroll
+  for (int nn = 0; nn < NH; ++nn) {
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o_acc[t][nn][e] = 0.f;
+    m_w[nn][0] = m_w[nn][1] = -INFINITY;
+    l_w[nn][0] = l_w[nn][1] = 0.f;
+  }
+
+  if (!r.dead && n > 0 && !failed) {
+    // ---- the earlier splits' maxima (lane x waits for split x) ----
+    float m_run = -INFINITY;   // warp 0, head lane: the running max entering the next tile
+    bool all_skipped = true;
+    if (ln.w == 0) {
+      float v[kMaxGroup];
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) v[h] = -INFINITY;
+      bool got = true;
+      if (ln.lane < split) {
+        const uint64_t t0 = globaltimer_ns();
+        for (int h = 0; h < G; ++h) {
+          unsigned long long w = 0;
+          for (uint32_t it = 0;; ++it) {
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(pub + ln.lane * G + h) : "memory");
+            if ((w >> 32) != 0ull) break;
+            if (it >= kSpinLimit || globaltimer_ns() - t0 > 1000000000ull) {
+              got = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+          if (!got) break;
+          const float x = __uint_as_float((uint32_t)w);
+#pragma unroll
+          for (int hh = 0; hh < kMaxGroup; ++hh)
+            if (hh == h) v[hh] = x;
+        }
+      }
+      if (!__all_sync(0xffffffffu, got)) {
+        if (ln.lane == 0) raise_error(p.err, ATTN_DEVERR_TIMEOUT);
+        failed = true;
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) {
+        if (h >= G) break;
+        const float mp = warp_max(v[h]);
+        if (ln.lane == h) m_run = mp;
+      }
+      // every tile of the split is skipped when its maximum is below the
+      // threshold against the earlier splits' for every head
+      all_skipped = __all_sync(0xffffffffu, ln.lane >= G || own == -INFINITY || own - m_run < p.thr_log2);
+    }
+    failed = __syncthreads_or(failed);
+    if (!failed && __syncthreads_and(all_skipped)) {
+      const int t0 = 2 * r.c0, t1 = min((r.L + kSkipTile - 1) / kSkipTile, 2 * r.c1);
+      if (tid == 0 && t1 > t0) {
+        if (p.skip_counts) {
+          atomicAdd(p.skip_counts + 0, (unsigned long long)(t1 - t0));
+          atomicAdd(p.skip_counts + 1, (unsigned long long)(t1 - t0));
+        }
+        if (p.skip_mask)
+          or_bit_range(p.skip_mask, (long long)seq * p.kt_max + t0, (long long)seq * p.kt_max + t1);
+      }
+      if (tid < G) {
+        const size_t row = ((size_t)b * p.h_q + (size_t)hk * G + tid) * kDecodeSplits + split;
+        p.ws_ml[row * 2 + 0] = -INFINITY;
+        p.ws_ml[row * 2 + 1] = 0.f;
+      }
+      return;
+    }
+
+    // ---- second half: the kept tiles' P.V (V chunks through the same ring) ----
+    if (!failed) {
+      const bool head = ln.lane < G;
+      unsigned long long n_vis = 0, n_skip = 0;
+      auto decide = [&](int c) -> uint32_t {
+        uint32_t kb = 0;
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const int tile = 2 * (r.c0 + c) + tt;
+          const bool vis = tile * kSkipTile < r.L;
+          const float tmv = (vis && head) ? tm_s[(2 * c + tt) * G + ln.lane] : -INFINITY;
+          // a head votes skip when exp(tile max - running max) < threshold
+          const bool vote = !head || tmv == -INFINITY || (tmv - m_run < p.thr_log2);
+          m_run = fmaxf(m_run, tmv);
+          const bool kept = vis && !__all_sync(0xffffffffu, vote);
+          if (kept) kb |= 1u << tt;
+          if (vis) {
+            ++n_vis;
+            if (!kept) {
+              ++n_skip;
+              if (p.skip_mask && ln.lane == 0) {
+                const long long unit = (long long)seq * p.kt_max + tile;
+                atomicOr(p.skip_mask + (unit >> 5), 1u << (unit & 31));
+              }
+            }
+          }
+        }
+        return kb;
+      };
+      // ring positions continue after the n K chunks
+      auto issue_v = [&](int i, int c, uint32_t kb) {   // lane 0 of warp 0
+        const int pos = n + i, st = pos % S;
+        const int tok0 = (r.c0 + c) * kChunk;
+        const int npg = (min(r.L - tok0, kChunk) + kPageSize - 1) / kPageSize;
+        // pages 0-1 hold tile A, 2-3 tile B
+        const int lo = (kb & 1u) ? 0 : ((kb & 2u) ? 2 : 4);
+        const int hi = min(npg, (kb & 2u) ? 4 : ((kb & 1u) ? 2 : 0));
+        keep_s[st] = kb;
+        keep_s[S + st] = (uint32_t)c;
+        mbar_arrive_expect_tx(&full[st], max(0, hi - lo) * (D / 64) * (16 * 64 * 2));
+        issue_pages<D>(&vmap, base + st * kSlot, &full[st], r.pages, tok0, r.L, hk, lo, hi, false);
+      };
+      // warp 0 decides the chunks in tile order and rings only the kept ones,
+      // the last marked (it decides one kept chunk ahead); a split with none
+      // kept gets one end entry
+      constexpr uint32_t kLast = 4u, kEndEntry = 0xffffffffu;
+      int next_c = 0, pend_c = 0;
+      uint32_t pend_kb = 0;
+      bool more = true;
+      auto find_kept = [&]() {
+        pend_kb = 0;
+        while (pend_kb == 0 && next_c < n) {
+          pend_c = next_c++;
+          pend_kb = decide(pend_c);
+        }
+      };
+      auto next_issue = [&](int i) {
+        const int c = pend_c;
+        const uint32_t kb = pend_kb;
+        if (kb) find_kept();
+        if (ln.lane == 0) {
+          if (kb) {
+            issue_v(i, c, kb | (pend_kb ? 0u : kLast));
+          } else {
+            keep_s[(n + i) % S] = kEndEntry;
+            mbar_arrive(&full[(n + i) % S]);
+          }
+        }
+        more = kb != 0 && pend_kb != 0;
+      };
+      int issued = 0;
+      if (ln.w == 0) {
+        find_kept();
+        for (; more && issued < S; ++issued) next_issue(issued);
+      }
+      for (int i = 0;; ++i) {
+        const int pos = n + i, st = pos % S;
+        const bool ok = mbar_wait(&full[st], (pos / S) & 1, p.err);
+        bool ended = false;
+        if (ok) {
+          const uint32_t kb = keep_s[st];
+          ended = kb == kEndEntry || (kb & kLast);
+          const int c = (int)keep_s[S + st];
+          const int tok_base = (r.c0 + c) * kChunk + ln.w * 16;
+          if (kb != kEndEntry && ((kb >> (ln.w >> 1)) & 1u) && tok_base < r.L) {
+            const uint32_t vslot = sbase + st * kSlot;
+            const float *ss = sc_s + (size_t)c * kChunk * G;
+            float sc[NH][4], qm[NH][2];
+#pragma unroll
+            for (int nn = 0; nn < NH; ++nn) {
+              qm[nn][0] = qm[nn][1] = -INFINITY;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int tl = ln.w * 16 + ln.g + 8 * (e >> 1);
+                const int h = 8 * nn + ln.cq + (e & 1);
+                const float v = (tok_base - ln.w * 16 + tl < r.L && h < G) ? ss[tl * G + h] : -INFINITY;
+                sc[nn][e] = v;
+                qm[nn][e & 1] = fmaxf(qm[nn][e & 1], v);
+              }
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1)
+                  qm[nn][h] = fmaxf(qm[nn][h], __shfl_xor_sync(0xffffffffu, qm[nn][h], o));
+            }
+            zero_tail_rows<D>(base, vslot, tok_base, r.L, ln);
+            warp_pv<D, NH>(o_acc, m_w, l_w, sc, qm, vslot, ln);
+          }
+        }
+        if (__syncthreads_or(!ok)) {
+          failed = true;
+          break;
+        }
+        if (ended) break;
+        // every warp is done with stage st
+        if (ln.w == 0 && more) {
+          next_issue(issued);
+          ++issued;
+        }
+      }
+      if (failed && tid == 0)
+        for (int x = issued - min(S, issued); x < issued; ++x)
+          mbar_wait(&full[(n + x) % S], ((n + x) / S) & 1, nullptr);
+      if (tid == 0 && p.skip_counts) {
+        atomicAdd(p.skip_counts + 0, n_vis);
+        atomicAdd(p.skip_counts + 1, n_skip);
+      }
+      __syncthreads();
+    }
+  }
+  merge_and_store<D, NH>(base, o_acc, m_w, l_w, r.dead || failed, G, b, hk, split, kDecodeSplits, false, p,
+                         ln);
+}
+
 // One warp per (sequence, q-head): log-sum-exp combine of the 32 split partials.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
@@ -1235,10 +1575,30 @@ cudaError_t launch_two_pass_g(const DecodeParams &p, const CUtensorMap &kmap, co
                       : launch_two_pass<D, 2, QDQ>(p, kmap, vmap, stream);
 }
 
+template <int D, int NH>
+cudaError_t launch_one_pass(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                            cudaStream_t stream) {
+  const size_t smem = 1024 + OnePassLayout(D, p.group, p.split_keys).total;
+  cudaError_t e = cudaFuncSetAttribute(decode_one_pass_kernel<D, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((long long)p.batch * p.h_kv * kDecodeSplits);
+  decode_one_pass_kernel<D, NH><<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_d(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
   const bool qdq = p.p_qdq || p.v_qdq;
+  if (p.sequential == 3) {
+    const cudaError_t e1 = p.group <= 8 ? launch_one_pass<D, 1>(p, kmap, vmap, stream)
+                                        : launch_one_pass<D, 2>(p, kmap, vmap, stream);
+    if (e1 != cudaSuccess) return e1;
+    const long long rows = (long long)p.batch * p.h_q;
+    decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
   if (p.sequential == 1)
     return qdq ? launch_g<D, true, true>(p, kmap, vmap, stream) : launch_g<D, true, false>(p, kmap, vmap, stream);
   cudaError_t e = p.sequential == 2
@@ -1252,6 +1612,14 @@ cudaError_t launch_d(const DecodeParams &p, const CUtensorMap &kmap, const CUten
 }
 
 }  // namespace
+
+size_t decode_one_pass_smem(int d, int group, int split_keys) {
+  const size_t bytes = 1024 + OnePassLayout(d, group, split_keys).total;
+  // the second half's merge reuses the ring and the scores
+  const size_t merge = (size_t)kWarps * 16 * 4 * 2 + (size_t)kWarps * 16 * d * 4;
+  if (OnePassLayout(d, group, split_keys).tm < merge) return 0;
+  return bytes <= 112 * 1024 ? bytes : 0;   // at least two CTAs per SM
+}
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream) {

@@ -53,13 +53,21 @@ struct DecodeParams {
   float *ws_s;                  // [B, h_kv, max_pages * 16, G] scores (two-pass skip)
   float *ws_tmax;               // [B, h_kv, kt_max, G] 32-key tile maxima (two-pass skip)
   float *ws_smax;               // [B, h_kv, splits, G] split maxima (two-pass skip)
+  // one-pass skip schedule: [B, h_kv, splits, G] published split maxima (high
+  // word 1 once written, low word the fp32 bits; zeroed before the launch),
+  // the launch's work-ticket counter (zeroed before the launch), and the most
+  // keys a split holds (its scores stay in shared memory)
+  unsigned long long *ws_pub;
+  unsigned int *ws_ticket;
+  int split_keys;
   uint32_t *skip_mask;          // or null
   unsigned long long *skip_counts;  // or null
   int batch, h_q, h_kv, group, d, num_pages, max_pages, kt_max;
   int s_stride;                 // key slots per (sequence, kv-head) in ws_s: max_pages * 16 rounded up to 64
   float scale_log2;             // scale * log2(e)
   float thr_log2;               // log2(threshold); -inf when skipping is off
-  int sequential;               // skip mode: 1 = one split walking 32-key tiles, 2 = two passes
+  int sequential;               // skip mode: 1 = one split walking 32-key tiles, 2 = two passes,
+                                // 3 = one pass over the splits (each waits for the earlier splits' maxima)
   // NVFP4 quantise-dequantise of P and / or V (skip schedules only): which
   // operands, their 448 / amax, their ratio tables g / (1 + j / 8), j = 0..7
   // (g = 2688 / amax, fp32), and the output factor 1 / g over the quantised
@@ -100,6 +108,9 @@ cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &qmap, const C
 cudaError_t launch_smallseq_bwd(const SmallSeqParams &p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);
+// Shared memory of the one-pass skip schedule for splits of up to `split_keys`
+// keys and groups of `group` heads (0 when it does not fit one CTA).
+size_t decode_one_pass_smem(int d, int group, int split_keys);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &qmap,
                            const CUtensorMap &kmap, const CUtensorMap &vmap, const CUtensorMap &omap,
                            cudaStream_t stream);

@@ -281,7 +281,10 @@ ATTN_API size_t attn_paged_decode_workspace_size(int batch, int h_q, int d);
  * skip_threshold > 0 gives the two-pass skip schedule's need: the split
  * partials plus, in float32, the scores of every (query head, key slot up to
  * max_pages_per_seq * 16, rounded up to 64), the maxima of every 32-key tile
- * and of every split (about batch * h_q * max_pages_per_seq * 64 bytes).
+ * and of every split (about batch * h_q * max_pages_per_seq * 64 bytes).  The
+ * one-pass form of that schedule uses the same workspace (the partials, and
+ * at the start of the scores area a work counter and the published split
+ * maxima, zeroed by the call in its stream).
  */
 ATTN_API size_t attn_paged_decode_workspace_size_ex(int batch, int h_q, int d, int max_pages_per_seq,
                                                     float skip_threshold);
@@ -303,13 +306,19 @@ ATTN_API size_t attn_paged_decode_workspace_size_ex(int batch, int h_q, int d, i
  *                  > 0 (and <= 1): skip-softmax over 32-key tiles visited in
  *                  order; a tile is skipped when all h_q / h_kv query heads
  *                  of the group vote skip against the running max.  With a
- *                  workspace this runs as two passes over the split schedule
- *                  (scores and tile maxima, then the kept tiles' P V): a
- *                  skipped tile never raises the running max, so the max
- *                  entering a tile is the max of all earlier tiles and every
- *                  split takes the sequential walk's decisions.  With
+ *                  workspace this runs over the split schedule: a skipped
+ *                  tile never raises the running max, so the max entering a
+ *                  tile is the max of all earlier tiles, and a split that
+ *                  knows the earlier splits' maxima takes the sequential
+ *                  walk's decisions.  When a split's scores fit one CTA's
+ *                  shared memory (keys per split * h_q / h_kv * 4 bytes, with
+ *                  the rest of the CTA's state, within 112 KB) it is one
+ *                  pass: each split's CTA computes its scores, publishes its
+ *                  maximum, waits for the earlier splits' and copies the
+ *                  kept tiles' V; otherwise two passes (scores and tile
+ *                  maxima to the workspace, then the kept tiles' P V).  With
  *                  workspace NULL it runs as one sequential split per
- *                  (sequence, kv-head).  Both give the same decisions.
+ *                  (sequence, kv-head).  All give the same decisions.
  *   out            [batch, h_q, d] bf16
  *   lse            [batch, h_q] float32, may be NULL
  *   workspace      device buffer of >= attn_paged_decode_workspace_size_ex(
@@ -400,9 +409,9 @@ ATTN_API int attn_paged_decode_qdq(const attn_bf16 *q, const attn_bf16 *k_cache,
  *     returns ATTN_E_TOO_LARGE and launches nothing: the shape fits when
  *     32 * batch * h_q * (4 d + 8) bytes, with the two parts (outputs, then
  *     max and sum) each rounded up to 256, is at most 48 MiB, i.e.
- *     batch * h_q <= 3024 at d = 128 and <= 5957 at d = 64.  In skip mode the two-pass
- *     schedule runs when its workspace fits the array, the sequential one
- *     (no workspace) otherwise.
+ *     batch * h_q <= 3024 at d = 128 and <= 5957 at d = 64.  In skip mode the split
+ *     schedule (one or two passes) runs when its workspace fits the array,
+ *     the sequential one (no workspace) otherwise.
  *   - every GPU that loads the library reserves those 48 MiB until the
  *     process exits.
  *   - the first call on a device looks up the array's device address
