@@ -1,6 +1,7 @@
 """GPU parity: paged one-token decode (dense split-KV + combine, and the
-skip-softmax schedules: two passes over the splits, or one sequential split)
-against the oracle."""
+skip-softmax schedules: the split schedule in one pass or, when a split's
+scores do not fit one CTA, two passes; or one sequential split) against the
+oracle."""
 import numpy as np
 import pytest
 import torch
@@ -154,6 +155,19 @@ def test_schedules_agree(A, d):
             assert int(c1[1]) > 0
         assert torch.allclose(o1.float(), o2.float(), atol=2e-2, rtol=0)
         assert torch.allclose(l1, l2, atol=1e-3, rtol=0)
+
+
+@pytest.mark.parametrize("thr", [1e-2, 0.5])
+def test_split_schedule_two_pass_form(A, thr):
+    """A group of 16 heads with a 50 000-token sequence: a split's scores
+    (1664 keys x 16 heads in fp32, 104 KB) no longer fit one CTA, so the split
+    schedule runs as two passes for the whole batch; checked against the
+    oracle, skip sets included."""
+    data = _peaked([1, 33, 700, 3000, 50000], h_q=16, h_kv=1, d=64, seed=16)
+    vis, skipped = _check(A, data, thr)
+    assert vis > 0
+    if thr >= 0.5:
+        assert skipped > 0
 
 
 def test_skip_threshold_zero_is_dense(A):
