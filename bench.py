@@ -336,8 +336,9 @@ def main():
         ops.append(("smallseq", do_smallseq))
 
     if args.only in ("decode_skip", "decode_qdq"):
-        # the decode workload in skip mode (threshold 0.1), two passes over the
-        # splits; decode_qdq adds NVFP4 quantise-dequantise of P and V (amax 1)
+        # the decode workload in skip mode (threshold 0.1) over the split
+        # schedule (one pass; two with quantisation); decode_qdq adds NVFP4
+        # quantise-dequantise of P and V (amax 1)
         qkw = dict(p_qdq="nvfp4", p_qdq_amax=1.0, v_qdq="nvfp4", v_qdq_amax=1.0) if args.only == "decode_qdq" else {}
         dsk_ws = torch.empty(A.attn_paged_decode_workspace_size(dec_batch, 32, 128, dec["block_table"].shape[1], 0.1),
                              dtype=torch.uint8, device=dev)
@@ -617,7 +618,8 @@ def _skip_decode_sweep(A, torch, dev, sd, reps, pk, runs):
         res[str(key)] = {"ms": ms, "skipped_frac": frac, "visited_tiles": vis, "skipped_tiles": sk,
                          "gbs": alg / ms / 1e6, "frac_of_measured": alg / ms / 1e6 / pk["hbm"],
                          "schedule": "dense split-KV" if thr == 0 and not qdq else
-                         ("two passes over 32 splits" if sched == "split" else "one sequential split")}
+                         (("two passes over 32 splits" if qdq else "one pass over 32 splits, scores on chip")
+                          if sched == "split" else "one sequential split")}
         if qdq:
             res[str(key)]["qdq"] = f"NVFP4 P (amax {qdq[0]}) and V (amax {qdq[1]})"
     return res
@@ -628,8 +630,9 @@ def measure_skip(A, W, torch, dev, seed, pk, reps=3):
     attention-sink workload on the same shapes, on which most tiles pass the
     skip test (what skipping saves)."""
     thresholds = (0.0, 1e-3, 1e-2, 0.1)
-    # skip mode runs the two-pass schedule (workspace given); "0.1/sequential"
-    # is the one-split-per-(sequence, kv-head) schedule at the same threshold
+    # skip mode runs the split schedule (workspace given: one pass, or two with
+    # quantisation); "0.1/sequential" is the one-split-per-(sequence, kv-head)
+    # schedule at the same threshold
     runs = [(t, t, "split") for t in thresholds] + [("0.1/sequential", 0.1, "sequential")]
     # NVFP4 quantise-dequantise of P and V (amax 1 each, the page's usage example)
     runs += [(f"qdq/{t}", t, "split", (1.0, 1.0)) for t in thresholds]
