@@ -170,6 +170,30 @@ def test_split_schedule_two_pass_form(A, thr):
         assert skipped > 0
 
 
+def test_split_schedule_concurrent_streams(A):
+    """Skip-mode decodes over the split schedule on two streams at once, each
+    call with its own workspace: a call's work counter and published split
+    maxima are its own, so every result equals the same call run alone (the
+    kernels are deterministic: bit-equal outputs, masks and counts)."""
+    runs = [_peaked([700, 3000, 9000], seed=21), _peaked([64, 5000, 20000, 1], h_q=16, h_kv=4, seed=22)]
+    devs = [_dev(d) for d in runs]
+    ref = [_run(A, d, 0.05, t) for d, t in zip(runs, devs)]
+    torch.cuda.synchronize()
+    assert A.attn_get_last_device_error() == 0
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    got = []
+    for _ in range(4):
+        for d, t, s in zip(runs, devs, streams):
+            with torch.cuda.stream(s):
+                got.append(_run(A, d, 0.05, t))
+    torch.cuda.synchronize()
+    assert A.attn_get_last_device_error() == 0
+    for i, g in enumerate(got):
+        r = ref[i % 2]
+        for a, b in zip(g[:4], r[:4]):
+            assert torch.equal(a, b)
+
+
 def test_skip_threshold_zero_is_dense(A):
     data = _peaked([100, 1000])
     t = _dev(data)
