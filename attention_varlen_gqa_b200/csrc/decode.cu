@@ -1183,8 +1183,8 @@ struct OnePassLayout {
     ring = 0;
     sc = ring + kOneStages * slot;                                   // [split_keys][G] scores
     tm = sc + (((size_t)split_keys * group * 4 + 15) & ~size_t(15)); // [split_keys / 32][G] tile maxima
-    qx = tm + (((size_t)(split_keys / kSkipTile) * group * 4 + 15) & ~size_t(15));   // [2][warp][16]
-    bt = qx + 2 * kWarps * 16 * 4;                                   // block-table entries
+    qx = tm + (((size_t)(split_keys / kSkipTile) * group * 4 + 15) & ~size_t(15));   // [chunk][warp][16]
+    bt = qx + (size_t)(split_keys / kChunk) * kWarps * 16 * 4;       // block-table entries
     keep = bt + kOneBtCap * 4;                                       // [stage] bits, [stage] chunk
     bar = keep + 2 * kOneStages * 4;                                 // [stage] mbarriers
     total = bar + kOneStages * 8;
@@ -1258,8 +1258,8 @@ __global__ void __launch_bounds__(kThreads) decode_one_pass_kernel(const __grid_
             if (h < G) sc_s[((size_t)i * kChunk + tl) * G + h] = sc[nn][e];
           }
           if (ln.g == 0) {
-            qx[((i & 1) * kWarps + ln.w) * 16 + 8 * nn + ln.cq] = qm[nn][0];
-            qx[((i & 1) * kWarps + ln.w) * 16 + 8 * nn + ln.cq + 1] = qm[nn][1];
+            qx[(i * kWarps + ln.w) * 16 + 8 * nn + ln.cq] = qm[nn][0];
+            qx[(i * kWarps + ln.w) * 16 + 8 * nn + ln.cq + 1] = qm[nn][1];
           }
         }
       }
@@ -1267,16 +1267,21 @@ __global__ void __launch_bounds__(kThreads) decode_one_pass_kernel(const __grid_
         failed = true;
         break;
       }
-      // every warp is done with stage st; chunk i's 16-key maxima are visible
+      // every warp is done with stage st
       if (tid == 0 && issued < n) issue_k(issued++);
-      if (tid < 2 * G) {
-        const int tt = tid / G, h = tid % G;
-        const float *x = qx + (i & 1) * kWarps * 16;
+    }
+    // the 32-key tile maxima from the warps' 16-key ones, once every chunk is
+    // in (off the per-chunk path); written and read by warp 0 only
+    if (!failed && tid < 2 * G) {
+      const int tt = tid / G, h = tid % G;
+      for (int i = 0; i < n; ++i) {
+        const float *x = qx + i * kWarps * 16;
         const float tmv = fmaxf(x[(2 * tt) * 16 + h], x[(2 * tt + 1) * 16 + h]);
         tm_s[(2 * i + tt) * G + h] = tmv;
         smax = fmaxf(smax, tmv);
       }
     }
+    __syncwarp();
     if (failed && tid == 0)
       for (int x = issued - min(S, issued); x < issued; ++x) mbar_wait(&full[x % S], (x / S) & 1, nullptr);
   }
