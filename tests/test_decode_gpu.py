@@ -160,9 +160,9 @@ def test_schedules_agree(A, d):
 @pytest.mark.parametrize("thr", [1e-2, 0.5])
 def test_split_schedule_two_pass_form(A, thr):
     """A group of 16 heads with a 50 000-token sequence: a split's scores
-    (1664 keys x 16 heads in fp32, 104 KB) no longer fit one CTA, so the split
-    schedule runs as two passes for the whole batch; checked against the
-    oracle, skip sets included."""
+    (1664 keys x 16 heads in fp32, 104 KB) no longer fit the one-pass CTA, so
+    the split schedule runs as two passes for the whole batch; checked
+    against the oracle, skip sets included."""
     data = _peaked([1, 33, 700, 3000, 50000], h_q=16, h_kv=1, d=64, seed=16)
     vis, skipped = _check(A, data, thr)
     assert vis > 0

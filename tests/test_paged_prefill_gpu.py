@@ -75,8 +75,11 @@ def test_chunked_prefill(A, causal, d, heads):
 
 
 @pytest.mark.parametrize("thr", [1e-2, 0.1])
-def test_chunked_prefill_skip(A, thr):
-    data = W.paged_prefill([200, 77], [700, 333], h_q=4, h_kv=2, d=128, seed=32)
+@pytest.mark.parametrize("heads", [(4, 2), (3, 1)])
+def test_chunked_prefill_skip(A, thr, heads):
+    """Skip mode on the paged cache; with a group of 3 an item's two query
+    blocks (one head) end one key tile apart."""
+    data = W.paged_prefill([200, 77], [700, 333], h_q=heads[0], h_kv=heads[1], d=128, seed=32)
     _check(A, data, True, thr)
 
 

@@ -124,6 +124,16 @@ def test_skip_sets(A, thr):
         assert skipped > 0
 
 
+@pytest.mark.parametrize("thr", [1e-2, 0.5])
+def test_skip_sets_odd_group(A, thr):
+    """Groups of 3 query heads: a work item is two consecutive query blocks of
+    one head, whose causal key ranges end one tile apart, so one tile of the
+    item stops a step early while the other's steps still skip."""
+    data = W.skip_parity_prefill([700, 300, 129], h_q=3, h_kv=1, d=128, seed=5)
+    vis, skipped = _check_full(A, data, thr)
+    assert vis > 0 and skipped > 0
+
+
 def test_skip_threshold_zero_equals_dense(A):
     data = W.skip_parity_prefill([400, 250], h_q=4, h_kv=2, d=64, seed=3)
     t = _dev(data)
