@@ -1623,7 +1623,9 @@ size_t decode_one_pass_smem(int d, int group, int split_keys) {
   // the second half's merge reuses the ring and the scores
   const size_t merge = (size_t)kWarps * 16 * 4 * 2 + (size_t)kWarps * 16 * d * 4;
   if (OnePassLayout(d, group, split_keys).tm < merge) return 0;
-  return bytes <= 112 * 1024 ? bytes : 0;   // at least two CTAs per SM
+  // four CTAs per SM (the occupancy it was measured at; with fewer, more of
+  // each CTA's per-chunk latency shows)
+  return bytes <= 56 * 1024 ? bytes : 0;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,

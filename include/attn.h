@@ -312,8 +312,8 @@ ATTN_API size_t attn_paged_decode_workspace_size_ex(int batch, int h_q, int d, i
  *                  knows the earlier splits' maxima takes the sequential
  *                  walk's decisions.  When a split's scores fit one CTA's
  *                  shared memory (keys per split * h_q / h_kv * 4 bytes, with
- *                  the rest of the CTA's state, within 112 KB) it is one
- *                  pass: each split's CTA computes its scores, publishes its
+ *                  the rest of the CTA's state, within 56 KB, so that four
+ *                  CTAs share an SM) it is one pass: each split's CTA computes its scores, publishes its
  *                  maximum, waits for the earlier splits' and copies the
  *                  kept tiles' V; otherwise two passes (scores and tile
  *                  maxima to the workspace, then the kept tiles' P V).  With
