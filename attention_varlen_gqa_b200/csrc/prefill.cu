@@ -720,7 +720,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // the V slot is released only after its copy has landed, read or not
-        if (ok && !v_ready) ok = wait_all(&v_full[st], (c / kStages) & 1);
+        if constexpr (SKIP) {
+          if (ok && !v_ready) ok = wait_all(&v_full[st], (c / kStages) & 1);
+        }
         if (ok) {
           // this tile's V, and the next tile's K once both S were issued above
           commit(&v_empty[st]);
